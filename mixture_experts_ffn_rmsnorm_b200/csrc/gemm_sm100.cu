@@ -1,0 +1,418 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// The grouped up- and down-projections of the routed experts (MoeLayer,
+// `forward_prefill`: sort-by-expert, then a tensor-core GEMM per expert with
+// each expert's weights loaded once), run together with a dense "class" of
+// tiles in the same launch (the always-on shared expert, nemotron_moe.rs
+// `prefill`, or LatentMoE fc1 / fc2), and the router GEMM with the sigmoid
+// top-k routing fused into its epilogue.
+//
+// Structure (one CTA per SM, persistent over a static round-robin tile list):
+//   warp 0   one lane issues TMA loads of A (128 x 128 B) and B (BN x 128 B)
+//            K-blocks into a STAGES-deep shared-memory ring (128-byte swizzle);
+//   warp 1   owns TMEM (2 x BN fp32 columns = two accumulators) and one lane
+//            issues tcgen05.mma (M = 128, N = BN) per K-step, committing each
+//            stage back to the producer and each finished tile to the epilogue;
+//   warps 2-5 read the accumulator rows from TMEM (tcgen05.ld), apply the
+//            epilogue (relu^2, scales, top-k, blend) and store to global
+//            memory while the MMA warp fills the other accumulator.
+// Every wait is bounded: a timeout sets a status bit and the CTA winds down
+// (draining its own TMA loads and MMAs) instead of hanging.
+#include "moe_internal.h"
+#include "ptx.cuh"
+#include "topk.cuh"
+
+namespace moe {
+namespace {
+
+template <int BN, int STAGES, bool FP8>
+struct Traits {
+  static constexpr int kBK = FP8 ? 128 : 64;        // K elements per stage (128 bytes)
+  static constexpr int kABytes = kBM * 128;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kUmmaK = FP8 ? 32 : 16;      // K per tcgen05.mma (32 bytes)
+  static constexpr int kKSteps = kBK / kUmmaK;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kSmem = STAGES * kStageBytes + 1024 + 256;
+  static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
+};
+
+struct Tile {
+  int c;        // class
+  int e;        // group (expert) index
+  int row0;     // first A row
+  int row_end;  // first A row not stored
+  int n0;       // first output column
+  int brow;     // first B row
+};
+
+template <int BN>
+__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w, int W0) {
+  Tile t;
+  if (w < W0) {
+    const int nt = p.cls[0].ntiles;
+    const int mt = w / nt;
+    const int ni = w - mt * nt;
+    t.c = 0;
+    if (p.tile_table) {
+      const int2 te = p.tile_table[mt];
+      t.e = te.x;
+      t.row0 = te.y;
+      t.row_end = p.group_off[te.x + 1];
+    } else {
+      t.e = 0;
+      t.row0 = mt * kBM;
+      t.row_end = p.cls[0].rows;
+    }
+    t.n0 = ni * BN;
+  } else {
+    w -= W0;
+    const int nt = p.cls[1].ntiles;
+    const int mt = w / nt;
+    const int ni = w - mt * nt;
+    t.c = 1;
+    t.e = 0;
+    t.row0 = mt * kBM;
+    t.row_end = p.cls[1].rows;
+    t.n0 = ni * BN;
+  }
+  t.brow = t.e * p.cls[t.c].N + t.n0;
+  return t;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+    u.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+    u.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+    u.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+    d[i] = u;
+  }
+}
+
+__device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort) {
+  *abort = 1;
+  if (p.status) atomicOr(p.status, kStatusWaitTimeout);
+}
+
+template <int BN, int STAGES, bool FP8>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using Tr = Traits<BN, STAGES, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* tiles = smem_raw + pad;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + STAGES * Tr::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA[0]);
+    tma_prefetch_desc(&p.tmB[0]);
+    if (p.nclasses > 1) {
+      tma_prefetch_desc(&p.tmA[1]);
+      tma_prefetch_desc(&p.tmB[1]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Tr::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m0 = p.n_mtiles ? *p.n_mtiles : p.cls[0].mtiles;
+  const int W0 = m0 * p.cls[0].ntiles;
+  const int W1 = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
+  const int W = W0 + W1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < W && ok; w += gridDim.x) {
+        const Tile t = decode_tile<BN>(p, w, W0);
+        const GemmClass& C = p.cls[t.c];
+        const int nk = (C.K + Tr::kBK - 1) / Tr::kBK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) {
+            record_timeout(p, abort);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = tiles + stage * Tr::kStageBytes;
+          uint8_t* sb = sa + Tr::kABytes;
+          mbar_arrive_expect_tx(&full[stage], Tr::kStageBytes);
+          const int kx = kb * Tr::kBK;
+          const int kbx = C.b_kwrap ? (kx % C.b_kwrap) : kx;
+          tma_load_2d(sa, &p.tmA[t.c], &full[stage], kx, t.row0);
+          tma_load_2d(sb, &p.tmB[t.c], &full[stage], kbx, t.brow);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the loads this thread issued land before the CTA exits: wait
+        // (bounded, ignoring the abort flag) on the last min(issued, STAGES)
+        // full barriers.
+        int s = stage;
+        uint32_t ph = phase;
+        const int n = issued < STAGES ? issued : STAGES;
+        for (int i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = STAGES - 1;
+            ph ^= 1u;
+          }
+          int zero = 0;
+          mbar_wait(&full[s], ph, &zero);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = FP8 ? make_idesc(kBM, BN, 0, 0) : make_idesc(kBM, BN, 1, 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < W && ok; w += gridDim.x, ++it) {
+        const Tile t = decode_tile<BN>(p, w, W0);
+        const int nk = (p.cls[t.c].K + Tr::kBK - 1) / Tr::kBK;
+        const int ab = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[ab], aph ^ 1u, abort)) {
+          record_timeout(p, abort);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + uint32_t(ab * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort)) {
+            record_timeout(p, abort);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* sa = tiles + stage * Tr::kStageBytes;
+          const uint64_t ad = smem_desc_sw128(sa);
+          const uint64_t bd = smem_desc_sw128(sa + Tr::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < Tr::kKSteps; ++kk) {
+            const uint64_t koff = uint64_t((kk * 32) >> 4);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            if (FP8)
+              umma_f8(d, ad + koff, bd + koff, idesc, acc);
+            else
+              umma_f16(d, ad + koff, bd + koff, idesc, acc);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit(&tfull[ab]);
+      }
+      // All MMAs this thread issued have completed once `drain` flips.
+      umma_commit(drain);
+      int zero = 0;
+      mbar_wait(drain, 0, &zero);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int rloc = q * 32 + lane;
+    int it = 0;
+    for (int w = blockIdx.x; w < W; w += gridDim.x, ++it) {
+      const Tile t = decode_tile<BN>(p, w, W0);
+      const GemmClass& C = p.cls[t.c];
+      const int ab = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!mbar_wait(&tfull[ab], aph, abort)) {
+        record_timeout(p, abort);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(ab * BN);
+      const int row = t.row0 + rloc;
+      const bool rvalid = row < t.row_end;
+
+      if (C.epi == EPI_TOPK) {
+        // Sigmoid top-k of one token (row) over E <= BN logits.
+        TopK tk;
+        tk.init();
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tb + uint32_t(c * 32), r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int e = c * 32 + j;
+            if (e < p.num_experts)
+              tk.offer(e, __uint_as_float(r[j]), p.gate_bias ? p.gate_bias[e] : 0.0f, p.top_k);
+          }
+        }
+        if (rvalid)
+          tk.write(p.top_k, p.rsf, p.topk_idx + size_t(row) * p.top_k,
+                   p.topk_w + size_t(row) * p.top_k);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tb + uint32_t(c * 32), r);
+          tmem_ld_wait();
+          const int n = t.n0 + c * 32;
+          if (rvalid && n < C.N) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (C.col_scale) {
+              const float4* cs =
+                  reinterpret_cast<const float4*>(C.col_scale + size_t(t.e) * C.N + n);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 s4 = cs[j];
+                v[4 * j + 0] *= s4.x;
+                v[4 * j + 1] *= s4.y;
+                v[4 * j + 2] *= s4.z;
+                v[4 * j + 3] *= s4.w;
+              }
+            }
+            if (C.row_scale) {
+              const float rs = C.row_scale[row];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= rs;
+            }
+            if (C.epi == EPI_RELU2_BF16) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = v[j] > 0.f ? v[j] * v[j] : 0.f;
+            }
+            if (C.epi == EPI_F32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(C.out) +
+                                                      size_t(row) * C.ldo + n);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            } else {
+              if (C.epi == EPI_BLEND) {
+                const float4* s4 =
+                    reinterpret_cast<const float4*>(p.blend_s + size_t(row) * C.ldo + n);
+                const uint4* r4 =
+                    reinterpret_cast<const uint4*>(p.blend_res + size_t(row) * C.ldo + n);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float4 a = s4[j];
+                  v[4 * j + 0] += a.x;
+                  v[4 * j + 1] += a.y;
+                  v[4 * j + 2] += a.z;
+                  v[4 * j + 3] += a.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint4 u = r4[j];
+                  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                  for (int h = 0; h < 4; ++h) {
+                    v[8 * j + 2 * h] += __uint_as_float(w4[h] << 16);
+                    v[8 * j + 2 * h + 1] += __uint_as_float(w4[h] & 0xFFFF0000u);
+                  }
+                }
+              }
+              store_bf16x32(static_cast<__nv_bfloat16*>(C.out) + size_t(row) * C.ldo + n, v);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Tr::kTmemCols);
+  }
+}
+
+template <int BN, int STAGES, bool FP8>
+cudaError_t launch_impl(const GemmParams& p, int grid, cudaStream_t stream) {
+  using Tr = Traits<BN, STAGES, FP8>;
+  auto kern = grouped_gemm_kernel<BN, STAGES, FP8>;
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kGemmThreads, Tr::kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int BN, int STAGES, bool FP8>
+cudaError_t prepare_impl() {
+  using Tr = Traits<BN, STAGES, FP8>;
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, STAGES, FP8>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::kSmem);
+}
+
+}  // namespace
+
+cudaError_t prepare_grouped_gemm() {
+  cudaError_t e;
+  if ((e = prepare_impl<128, 6, false>()) != cudaSuccess) return e;
+  if ((e = prepare_impl<128, 6, true>()) != cudaSuccess) return e;
+  if ((e = prepare_impl<256, 4, false>()) != cudaSuccess) return e;
+  return prepare_impl<256, 4, true>();
+}
+
+cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, bool fp8, int grid,
+                                cudaStream_t stream) {
+  if (bn == 128) {
+    return fp8 ? launch_impl<128, 6, true>(p, grid, stream)
+               : launch_impl<128, 6, false>(p, grid, stream);
+  }
+  if (bn == 256) {
+    return fp8 ? launch_impl<256, 4, true>(p, grid, stream)
+               : launch_impl<256, 4, false>(p, grid, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,543 @@
+// C ABI of the MoE FFN layer (include/moe_b200.h): argument validation,
+// workspace, TMA descriptors and the launch sequence of both paths.
+//
+// Prefill path (any T), after NemotronMoeLayer `prefill` and MoeLayer
+// `forward_prefill`:
+//   rmsnorm -> router GEMM with fused sigmoid top-k (+ LatentMoE fc1 in the
+//   same launch) -> sort by expert -> gather -> grouped up GEMM + relu^2
+//   (routed experts and shared expert in one launch) -> grouped down GEMM
+//   (routed + shared) -> unpermute + weighted reduce + shared + residual
+//   (direct) or latent reduce -> fc2 GEMM with shared + residual blend.
+// Decode path (T <= 8): decode.cu.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/moe_b200.h"
+#include "decode.h"
+#include "moe_internal.h"
+
+using moe::GemmParams;
+using bf16 = __nv_bfloat16;
+
+namespace {
+
+constexpr uint32_t kMagic = 0x4D6F4542u;  // "MoEB"
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D K-major operand map: inner = K extent (elements), rows, row stride in
+// bytes; box = 128 bytes of K x box_rows rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner, uint64_t rows,
+              uint64_t row_stride_bytes, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {byte_elems ? 128u : 64u, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, byte_elems ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+struct moe_handle {
+  uint32_t magic;
+  moe_config cfg;
+  moe_weights w;
+  int device;
+  int num_sms;
+  int D;           // routed-expert width
+  bool fp8;
+  int gate_bn;     // router GEMM tile width (>= E)
+  int last_launches;
+  int last_tokens;    // num_tokens of the last forward
+  bool last_decode;   // whether it took the decode path
+  // workspace
+  void* ws;
+  size_t ws_bytes;
+  bf16* gate_a;    // [Tm, 2H]: normed bf16 (hi) | residual of the rounding (lo)
+  int32_t* idx;    // [Tm*k]
+  float* wts;      // [Tm*k]  (immediately after idx, as the pages' scratch layout)
+  int32_t* off;    // [E+1]
+  int2* tiles;     // [Rm/128 + E]
+  int32_t* n_mtiles;
+  int32_t* status;
+  int32_t* perm;   // [Rm]
+  int32_t* inv;    // [Rm]
+  bf16* z;         // [Tm, L]   latent fc1 output
+  bf16* xs;        // [Rm, D]   sorted expert inputs
+  bf16* u;         // [Rm, I]   relu^2(up)
+  bf16* v;         // [Tm, S]   shared relu^2(up)
+  bf16* y;         // [Rm, D]   routed expert outputs (sorted order)
+  float* s;        // [Tm, H]   shared expert output
+  bf16* m;         // [Tm, L]   latent weighted sum
+  bf16* stage_h;   // [Tm, H]   host-path staging
+  bf16* stage_r;   // [Tm, H]
+  moe::DecodeWorkspace dec;
+  // tensor maps
+  CUtensorMap tm_gate_a, tm_gate_b, tm_fc1_a, tm_fc1_b;
+  CUtensorMap tm_up_a, tm_up_b, tm_sup_a, tm_sup_b;
+  CUtensorMap tm_down_a, tm_down_b, tm_sdown_a, tm_sdown_b;
+  CUtensorMap tm_fc2_a, tm_fc2_b;
+};
+
+namespace {
+
+moe_status check_handle(const moe_handle* h) {
+  return (h && h->magic == kMagic) ? MOE_OK : MOE_ERR_INVALID_HANDLE;
+}
+
+moe_status validate_config(const moe_config* c) {
+  if (c->hidden_size <= 0 || c->num_experts <= 0 || c->moe_inter <= 0 || c->shared_inter <= 0 ||
+      c->latent_size < 0 || c->max_tokens < 1)
+    return MOE_ERR_INVALID_CONFIG;
+  if (c->top_k < 1 || c->top_k > c->num_experts || c->top_k > MOE_MAX_TOP_K ||
+      c->num_experts > MOE_MAX_EXPERTS)
+    return MOE_ERR_INVALID_CONFIG;
+  if (c->hidden_size % 64 || c->moe_inter % 64 || c->shared_inter % 64 || c->latent_size % 64)
+    return MOE_ERR_INVALID_CONFIG;
+  if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps) ||
+      !std::isfinite(c->routed_scaling_factor))
+    return MOE_ERR_INVALID_CONFIG;
+  if (c->expert_wdtype != MOE_WEIGHTS_BF16 && c->expert_wdtype != MOE_WEIGHTS_FP8_E4M3_ROWSCALE)
+    return MOE_ERR_INVALID_CONFIG;
+  // row counts of the stacked expert maps and tile tables must fit in int32
+  const long long D = c->latent_size ? c->latent_size : c->hidden_size;
+  const long long R = 1ll * c->max_tokens * c->top_k;
+  if (1ll * c->num_experts * c->moe_inter > (1ll << 31) - 1 ||
+      1ll * c->num_experts * D > (1ll << 31) - 1 || R * (D > c->moe_inter ? D : c->moe_inter) >
+                                                      (1ll << 40))
+    return MOE_ERR_INVALID_CONFIG;
+  return MOE_OK;
+}
+
+moe_status validate_weights(const moe_config* c, const moe_weights* w) {
+  const bool fp8 = c->expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE;
+  const void* req[] = {w->norm_w, w->gate_w, w->up_w, w->down_w, w->shared_up_w, w->shared_down_w};
+  for (const void* p : req)
+    if (!p) return MOE_ERR_NULL_POINTER;
+  if (fp8 && (!w->up_scale || !w->down_scale)) return MOE_ERR_NULL_POINTER;
+  if (c->latent_size > 0 && (!w->fc1_w || !w->fc2_w)) return MOE_ERR_NULL_POINTER;
+  const void* all[] = {w->norm_w, w->gate_w, w->gate_bias, w->up_w, w->down_w, w->up_scale,
+                       w->down_scale, w->shared_up_w, w->shared_down_w, w->fc1_w, w->fc2_w};
+  for (const void* p : all)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+struct Carver {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off = round_up(off + count * sizeof(T), 256);
+    return p;
+  }
+};
+
+void carve(moe_handle* h, char* base) {
+  const moe_config& c = h->cfg;
+  const size_t Tm = c.max_tokens, k = c.top_k, E = c.num_experts, H = c.hidden_size;
+  const size_t Rm = Tm * k, D = h->D, I = c.moe_inter, S = c.shared_inter, L = c.latent_size;
+  Carver cv{base};
+  h->gate_a = cv.take<bf16>(Tm * 2 * H);
+  h->idx = cv.take<int32_t>(Rm);
+  h->wts = cv.take<float>(Rm);
+  h->off = cv.take<int32_t>(E + 1);
+  h->tiles = cv.take<int2>(Rm / moe::kBM + E + 1);
+  h->n_mtiles = cv.take<int32_t>(1);
+  h->status = cv.take<int32_t>(1);
+  h->perm = cv.take<int32_t>(Rm);
+  h->inv = cv.take<int32_t>(Rm);
+  h->z = L ? cv.take<bf16>(Tm * L) : nullptr;
+  h->xs = cv.take<bf16>(Rm * D);
+  h->u = cv.take<bf16>(Rm * I);
+  h->v = cv.take<bf16>(Tm * S);
+  h->y = cv.take<bf16>(Rm * D);
+  h->s = cv.take<float>(Tm * H);
+  h->m = L ? cv.take<bf16>(Tm * L) : nullptr;
+  h->stage_h = cv.take<bf16>(Tm * H);
+  h->stage_r = cv.take<bf16>(Tm * H);
+  moe::carve_decode(&h->dec, c, [&](size_t bytes) { return cv.take<char>(bytes); });
+  h->ws_bytes = cv.off;
+}
+
+bool build_maps(moe_handle* h) {
+  const moe_config& c = h->cfg;
+  const uint64_t Tm = c.max_tokens, E = c.num_experts, H = c.hidden_size;
+  const uint64_t Rm = Tm * c.top_k, D = h->D, I = c.moe_inter, S = c.shared_inter,
+                 L = c.latent_size;
+  const bool f8 = h->fp8;
+  const uint64_t eb = f8 ? 1 : 2;  // bytes per routed-expert operand element
+  bool ok = true;
+  // router: A = [hi | lo] (K = 2H), B = gate [E, H] (k wraps at H)
+  ok &= make_map(&h->tm_gate_a, h->gate_a, false, 2 * H, Tm, 2 * H * 2, moe::kBM);
+  ok &= make_map(&h->tm_gate_b, h->w.gate_w, false, H, E, H * 2, h->gate_bn);
+  if (L) {
+    ok &= make_map(&h->tm_fc1_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
+    ok &= make_map(&h->tm_fc1_b, h->w.fc1_w, false, H, L, H * 2, h->gate_bn);
+    ok &= make_map(&h->tm_fc2_a, h->m, false, L, Tm, L * 2, moe::kBM);
+    ok &= make_map(&h->tm_fc2_b, h->w.fc2_w, false, L, H, L * 2, 128);
+  }
+  // grouped up: routed A = xs [Rm, D], B = up [E*I, D]; shared A = normed, B = [S, H]
+  ok &= make_map(&h->tm_up_a, h->xs, f8, D, Rm, D * eb, moe::kBM);
+  ok &= make_map(&h->tm_up_b, h->w.up_w, f8, D, E * I, D * eb, 128);
+  ok &= make_map(&h->tm_sup_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
+  ok &= make_map(&h->tm_sup_b, h->w.shared_up_w, false, H, S, H * 2, 128);
+  // grouped down: routed A = u [Rm, I], B = down [E*D, I]; shared A = v, B = [H, S]
+  ok &= make_map(&h->tm_down_a, h->u, f8, I, Rm, I * eb, moe::kBM);
+  ok &= make_map(&h->tm_down_b, h->w.down_w, f8, I, E * D, I * eb, 128);
+  ok &= make_map(&h->tm_sdown_a, h->v, false, S, Tm, S * 2, moe::kBM);
+  ok &= make_map(&h->tm_sdown_b, h->w.shared_down_w, false, S, H, S * 2, 128);
+  return ok;
+}
+
+moe::GemmClass dense_class(int K, int N, int rows, int epi, void* out, int ldo, int bn) {
+  moe::GemmClass c{};
+  c.K = K;
+  c.N = N;
+  c.ntiles = (N + bn - 1) / bn;
+  c.rows = rows;
+  c.mtiles = (rows + moe::kBM - 1) / moe::kBM;
+  c.epi = epi;
+  c.out = out;
+  c.ldo = ldo;
+  return c;
+}
+
+#define MOE_TRY(expr)                                  \
+  do {                                                 \
+    cudaError_t _e = (expr);                           \
+    if (_e != cudaSuccess) return MOE_ERR_CUDA;        \
+  } while (0)
+
+// Norm + router GEMM with fused top-k (+ fc1 for LatentMoE).
+moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int T,
+                         bool with_fc1, cudaStream_t st, int* launches) {
+  const moe_config& c = h->cfg;
+  MOE_TRY(moe::launch_rmsnorm(hidden, static_cast<const bf16*>(h->w.norm_w), residual, h->gate_a,
+                              T, c.hidden_size, c.rms_eps, st));
+  ++*launches;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.tmA[0] = h->tm_gate_a;
+  p.tmB[0] = h->tm_gate_b;
+  p.cls[0] = dense_class(2 * c.hidden_size, c.num_experts, T, moe::EPI_TOPK, nullptr, 0,
+                         h->gate_bn);
+  p.cls[0].ntiles = 1;
+  p.cls[0].b_kwrap = c.hidden_size;
+  p.nclasses = 1;
+  if (with_fc1 && c.latent_size > 0) {
+    p.tmA[1] = h->tm_fc1_a;
+    p.tmB[1] = h->tm_fc1_b;
+    p.cls[1] = dense_class(c.hidden_size, c.latent_size, T, moe::EPI_BF16, h->z, c.latent_size,
+                           h->gate_bn);
+    p.nclasses = 2;
+  }
+  p.gate_bias = h->w.gate_bias;
+  p.top_k = c.top_k;
+  p.num_experts = c.num_experts;
+  p.rsf = c.routed_scaling_factor;
+  p.topk_idx = h->idx;
+  p.topk_w = h->wts;
+  p.status = h->status;
+  int W = p.cls[0].mtiles + (p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0);
+  const int grid = W < h->num_sms ? W : h->num_sms;
+  MOE_TRY(moe::launch_grouped_gemm(p, h->gate_bn, false, grid, st));
+  ++*launches;
+  return MOE_OK;
+}
+
+moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, cudaStream_t st,
+                           int* launches) {
+  const moe_config& c = h->cfg;
+  const int H = c.hidden_size, k = c.top_k, E = c.num_experts, I = c.moe_inter,
+            S = c.shared_inter, L = c.latent_size, D = h->D, R = T * k;
+  moe_status rs = enqueue_route(h, hidden, residual, T, true, st, launches);
+  if (rs != MOE_OK) return rs;
+  MOE_TRY(moe::launch_sort(h->idx, T, k, E, h->perm, h->inv, h->off, h->tiles, h->n_mtiles,
+                           h->status, st));
+  ++*launches;
+  if (L)
+    MOE_TRY(moe::launch_gather(h->z, L, h->perm, k, R, D, h->xs, st));
+  else
+    MOE_TRY(moe::launch_gather(h->gate_a, 2 * H, h->perm, k, R, D, h->xs, st));
+  ++*launches;
+
+  // grouped up (+ relu^2): routed class 0 via the tile table, shared class 1
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.tmA[0] = h->tm_up_a;
+  p.tmB[0] = h->tm_up_b;
+  p.cls[0] = dense_class(D, I, 0, moe::EPI_RELU2_BF16, h->u, I, 128);
+  p.tmA[1] = h->tm_sup_a;
+  p.tmB[1] = h->tm_sup_b;
+  p.cls[1] = dense_class(H, S, T, moe::EPI_RELU2_BF16, h->v, S, 128);
+  p.nclasses = 2;
+  p.tile_table = h->tiles;
+  p.n_mtiles = h->n_mtiles;
+  p.group_off = h->off;
+  p.status = h->status;
+  MOE_TRY(moe::launch_grouped_gemm(p, 128, false, h->num_sms, st));
+  ++*launches;
+
+  // grouped down: routed -> y (bf16, sorted rows), shared -> s (f32)
+  p.tmA[0] = h->tm_down_a;
+  p.tmB[0] = h->tm_down_b;
+  p.cls[0] = dense_class(I, D, 0, moe::EPI_BF16, h->y, D, 128);
+  p.tmA[1] = h->tm_sdown_a;
+  p.tmB[1] = h->tm_sdown_b;
+  p.cls[1] = dense_class(S, H, T, moe::EPI_F32, h->s, H, 128);
+  MOE_TRY(moe::launch_grouped_gemm(p, 128, false, h->num_sms, st));
+  ++*launches;
+
+  if (!L) {
+    MOE_TRY(moe::launch_combine(h->y, h->inv, h->wts, h->s, residual, hidden, T, k, H, st));
+    ++*launches;
+    return MOE_OK;
+  }
+  MOE_TRY(moe::launch_latent_reduce(h->y, h->inv, h->wts, h->m, T, k, L, st));
+  ++*launches;
+  GemmParams q;
+  std::memset(&q, 0, sizeof(q));
+  q.tmA[0] = h->tm_fc2_a;
+  q.tmB[0] = h->tm_fc2_b;
+  q.cls[0] = dense_class(L, H, T, moe::EPI_BLEND, hidden, H, 128);
+  q.nclasses = 1;
+  q.blend_s = h->s;
+  q.blend_res = residual;
+  q.status = h->status;
+  const int W = q.cls[0].mtiles * q.cls[0].ntiles;
+  MOE_TRY(moe::launch_grouped_gemm(q, 128, false, W < h->num_sms ? W : h->num_sms, st));
+  ++*launches;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_CONFIG: return "invalid configuration";
+    case MOE_ERR_NULL_POINTER: return "required pointer is NULL";
+    case MOE_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case MOE_ERR_TOKENS_OUT_OF_RANGE: return "num_tokens outside [1, max_tokens]";
+    case MOE_ERR_OUT_OF_MEMORY: return "workspace allocation failed";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE: return "no sm_100 device is current";
+    case MOE_ERR_INVALID_HANDLE: return "invalid handle";
+  }
+  return "unknown status";
+}
+
+moe_status moe_create(const moe_config* config, const moe_weights* weights, moe_handle** out) {
+  if (!out) return MOE_ERR_NULL_POINTER;
+  *out = nullptr;
+  if (!config || !weights) return MOE_ERR_NULL_POINTER;
+  moe_status st = validate_config(config);
+  if (st != MOE_OK) return st;
+  st = validate_weights(config, weights);
+  if (st != MOE_OK) return st;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_DEVICE;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_DEVICE;
+  if (prop.major != 10) return MOE_ERR_DEVICE;
+
+  moe_handle* h = new (std::nothrow) moe_handle();
+  if (!h) return MOE_ERR_OUT_OF_MEMORY;
+  h->magic = kMagic;
+  h->cfg = *config;
+  h->w = *weights;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->D = config->latent_size ? config->latent_size : config->hidden_size;
+  h->fp8 = config->expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE;
+  h->gate_bn = config->num_experts <= 128 ? 128 : 256;
+  if (h->fp8) {  // the FP8 grouped GEMMs are not wired yet
+    delete h;
+    return MOE_ERR_INVALID_CONFIG;
+  }
+
+  carve(h, nullptr);
+  void* ws = nullptr;
+  if (cudaMalloc(&ws, h->ws_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MOE_ERR_OUT_OF_MEMORY;
+  }
+  h->ws = ws;
+  carve(h, static_cast<char*>(ws));
+  if (cudaMemset(ws, 0, h->ws_bytes) != cudaSuccess || !build_maps(h) ||
+      moe::prepare_grouped_gemm() != cudaSuccess || moe::prepare_decode() != cudaSuccess) {
+    cudaFree(ws);
+    h->magic = 0;
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_destroy(moe_handle* h) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != h->device) cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  cudaFree(h->ws);
+  if (cur != h->device) cudaSetDevice(cur);
+  h->magic = 0;
+  delete h;
+  return MOE_OK;
+}
+
+moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t num_tokens,
+                            int32_t path, void* stream) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  if (!hidden || !residual) return MOE_ERR_NULL_POINTER;
+  if (!aligned16(hidden) || !aligned16(residual)) return MOE_ERR_MISALIGNED;
+  if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL)
+    return MOE_ERR_INVALID_CONFIG;
+  if (path == MOE_PATH_DECODE && num_tokens > MOE_DECODE_MAX_TOKENS)
+    return MOE_ERR_TOKENS_OUT_OF_RANGE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  const bool decode = path == MOE_PATH_DECODE ||
+                      (path == MOE_PATH_AUTO && num_tokens <= MOE_DECODE_MAX_TOKENS &&
+                       moe::decode_supported(h->cfg));
+  if (decode) {
+    moe::DecodeArgs a;
+    a.cfg = &h->cfg;
+    a.w = &h->w;
+    a.ws = &h->dec;
+    a.status = h->status;
+    st = moe::enqueue_decode(a, static_cast<bf16*>(hidden), static_cast<bf16*>(residual),
+                             num_tokens, s, &launches);
+  } else {
+    st = enqueue_prefill(h, static_cast<bf16*>(hidden), static_cast<bf16*>(residual), num_tokens,
+                         s, &launches);
+  }
+  h->last_launches = launches;
+  h->last_tokens = num_tokens;
+  h->last_decode = decode;
+  return st;
+}
+
+moe_status moe_forward(moe_handle* h, void* hidden, void* residual, int32_t num_tokens,
+                       void* stream) {
+  return moe_forward_path(h, hidden, residual, num_tokens, MOE_PATH_AUTO, stream);
+}
+
+moe_status moe_forward_host(moe_handle* h, void* hidden_host, void* residual_host,
+                            int32_t num_tokens, void* stream) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  if (!hidden_host) return MOE_ERR_NULL_POINTER;
+  if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = size_t(num_tokens) * h->cfg.hidden_size * sizeof(bf16);
+  MOE_TRY(cudaMemcpyAsync(h->stage_h, hidden_host, bytes, cudaMemcpyHostToDevice, s));
+  st = moe_forward(h, h->stage_h, h->stage_r, num_tokens, stream);
+  if (st != MOE_OK) return st;
+  MOE_TRY(cudaMemcpyAsync(hidden_host, h->stage_h, bytes, cudaMemcpyDeviceToHost, s));
+  if (residual_host)
+    MOE_TRY(cudaMemcpyAsync(residual_host, h->stage_r, bytes, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+moe_status moe_route(moe_handle* h, const void* hidden, int32_t num_tokens, int32_t* idx,
+                     float* w, void* stream) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  if (!hidden || !idx || !w) return MOE_ERR_NULL_POINTER;
+  if (!aligned16(hidden)) return MOE_ERR_MISALIGNED;
+  if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  st = enqueue_route(h, static_cast<const bf16*>(hidden), h->stage_r, num_tokens, false, s,
+                     &launches);
+  if (st != MOE_OK) return st;
+  const size_t n = size_t(num_tokens) * h->cfg.top_k;
+  MOE_TRY(cudaMemcpyAsync(idx, h->idx, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  MOE_TRY(cudaMemcpyAsync(w, h->wts, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  h->last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_tokens, int32_t* perm,
+                    int32_t* inv, int32_t* off, void* stream) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  if (!idx || !perm || !inv || !off) return MOE_ERR_NULL_POINTER;
+  if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
+  MOE_TRY(moe::launch_sort(idx, num_tokens, h->cfg.top_k, h->cfg.num_experts, perm, inv, off,
+                           h->tiles, h->n_mtiles, h->status, static_cast<cudaStream_t>(stream)));
+  h->last_launches = 1;
+  return MOE_OK;
+}
+
+moe_status moe_copy_routing(moe_handle* h, int32_t* idx, float* w, int32_t num_tokens,
+                            void* stream) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  if (!idx || !w) return MOE_ERR_NULL_POINTER;
+  if (num_tokens < 1 || num_tokens != h->last_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t n = size_t(num_tokens) * h->cfg.top_k;
+  const int32_t* si = h->last_decode ? h->dec.idx : h->idx;
+  const float* sw = h->last_decode ? h->dec.w : h->wts;
+  MOE_TRY(cudaMemcpyAsync(idx, si, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  MOE_TRY(cudaMemcpyAsync(w, sw, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  return MOE_OK;
+}
+
+moe_status moe_get_device_status(moe_handle* h, int32_t* status, void* stream) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  if (!status) return MOE_ERR_NULL_POINTER;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(cudaMemcpyAsync(status, h->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  MOE_TRY(cudaMemsetAsync(h->status, 0, sizeof(int32_t), s));
+  MOE_TRY(cudaStreamSynchronize(s));
+  return MOE_OK;
+}
+
+int32_t moe_last_launch_count(const moe_handle* h) {
+  return check_handle(h) == MOE_OK ? h->last_launches : -1;
+}
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+// Internal declarations shared by the kernels and the C-ABI host code.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kBM = 128;             // GEMM tile rows (UMMA M)
+constexpr int kGemmThreads = 192;    // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
+constexpr int kMaxTopKShared = 16;   // top_k bound of the routing kernels
+
+// What the GEMM epilogue does with an accumulator row segment.
+enum EpiKind : int {
+  EPI_BF16 = 0,        // out = bf16(acc)
+  EPI_RELU2_BF16 = 1,  // out = bf16(max(acc, 0)^2)
+  EPI_F32 = 2,         // out = acc (float32)
+  EPI_TOPK = 3,        // sigmoid top-k routing of the row (gate logits never stored)
+  EPI_BLEND = 4,       // out = bf16(acc + blend_s + blend_res)  (LatentMoE fc2)
+};
+
+// One class of GEMM tiles inside a launch.  A is [rows, K] (K contiguous),
+// B is [groups * N, K]; a tile multiplies 128 rows of A by BN rows of one
+// group of B.
+struct GemmClass {
+  int K;                  // reduction length in elements
+  int N;                  // output columns of one group (B rows per group)
+  int ntiles;             // ceil(N / BN)
+  int mtiles;             // m-tiles of a dense class (ignored when the launch has a tile table)
+  int rows;               // valid A rows of a dense class
+  int b_kwrap;            // B's k coordinate is taken modulo this (0 = no wrap)
+  int epi;                // EpiKind
+  void* out;              // output base
+  int ldo;                // output row stride in elements
+  const float* col_scale; // [groups, N] per-output-column scale (FP8 weights) or null
+  const float* row_scale; // [rows] per-A-row scale or null
+};
+
+struct GemmParams {
+  CUtensorMap tmA[2];
+  CUtensorMap tmB[2];
+  GemmClass cls[2];
+  int nclasses;
+  // Grouped class 0: m-tile i covers sorted rows [tile_table[i].y, +128)
+  // of group tile_table[i].x; rows at or beyond group_off[x + 1] belong to the
+  // next group and are not stored.  n_mtiles is the device-side tile count.
+  const int2* tile_table;
+  const int* n_mtiles;
+  const int* group_off;
+  // EPI_TOPK
+  const float* gate_bias;
+  int top_k;
+  int num_experts;
+  float rsf;
+  int* topk_idx;
+  float* topk_w;
+  // EPI_BLEND
+  const float* blend_s;
+  const __nv_bfloat16* blend_res;
+  int* status;
+};
+
+// Launch the persistent grouped GEMM (bn = 128 or 256; fp8 = E4M3 operands).
+cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, bool fp8, int grid,
+                                cudaStream_t stream);
+// Set the dynamic shared memory limit of every GEMM instantiation on the
+// current device (call once per device before launching).
+cudaError_t prepare_grouped_gemm();
+
+// Routing / sort / data movement kernels (route.cu).
+cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* norm_w,
+                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, int T, int H,
+                           float eps, cudaStream_t stream);
+size_t sort_smem_bytes(int E);
+cudaError_t launch_sort(const int* idx, int T, int k, int E, int* perm, int* inv, int* off,
+                        int2* tile_table, int* n_mtiles, int* status, cudaStream_t stream);
+cudaError_t launch_gather(const __nv_bfloat16* X, int ldx, const int* perm, int k, int R, int D,
+                          __nv_bfloat16* xs, cudaStream_t stream);
+cudaError_t launch_combine(const __nv_bfloat16* y, const int* inv, const float* w,
+                           const float* s, const __nv_bfloat16* residual,
+                           __nv_bfloat16* hidden, int T, int k, int H, cudaStream_t stream);
+cudaError_t launch_latent_reduce(const __nv_bfloat16* y, const int* inv, const float* w,
+                                 __nv_bfloat16* m, int T, int k, int L, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,68 @@
+// Sigmoid top-k selection of one token, shared by the prefill router GEMM
+// epilogue and the decode routing kernel so both paths take identical
+// decisions in float32.
+//
+// NemotronMoeLayer (nemotron_moe.rs module documentation): sigmoid top-k
+// routing.  Selection key = sigmoid(logit) + bias (bias for selection only);
+// slots are kept in descending key order and a key only displaces strictly
+// smaller ones, so on equal keys the lower expert index (visited first) wins.
+// Weights: the unbiased scores of the selected experts renormalised to sum 1
+// and multiplied by routed_scaling_factor.
+#pragma once
+
+namespace moe {
+
+constexpr int kTopKMax = 16;
+
+struct TopK {
+  float key[kTopKMax];
+  float score[kTopKMax];
+  int id[kTopKMax];
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < kTopKMax; ++j) {
+      key[j] = -INFINITY;
+      score[j] = 0.f;
+      id[j] = -1;
+    }
+  }
+
+  // Offer expert e (experts must be offered in increasing index order).
+  __device__ __forceinline__ void offer(int e, float logit, float bias, int k) {
+    const float s = 1.0f / (1.0f + expf(-logit));
+    const float kk = s + bias;
+#pragma unroll
+    for (int x = kTopKMax - 1; x >= 0; --x) {
+      if (x < k && kk > key[x]) {
+        if (x > 0 && kk > key[x - 1]) {
+          key[x] = key[x - 1];
+          score[x] = score[x - 1];
+          id[x] = id[x - 1];
+        } else {
+          key[x] = kk;
+          score[x] = s;
+          id[x] = e;
+        }
+      }
+    }
+  }
+
+  // Renormalised weights times rsf into w[0..k), ids into idx[0..k).
+  __device__ __forceinline__ void write(int k, float rsf, int* idx, float* w) const {
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < kTopKMax; ++j)
+      if (j < k) sum += score[j];
+    const float scale = rsf / sum;
+#pragma unroll
+    for (int j = 0; j < kTopKMax; ++j) {
+      if (j < k) {
+        idx[j] = id[j];
+        w[j] = score[j] * scale;
+      }
+    }
+  }
+};
+
+}  // namespace moe

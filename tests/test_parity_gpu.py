@@ -1,0 +1,212 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Bars (from the layer's tolerance statement): sort / permutation / offsets
+bit-exact given the same routing; routing sets identical except where the
+oracle's k-th and (k+1)-th selection keys differ by less than 1e-5 (counted);
+layer output max|gpu - oracle| <= c * max|oracle| + 1e-3 with c = 1e-2 for
+BF16 expert weights and 5e-2 for FP8.  Full-size workloads are checked on
+sampled tokens (tokens are independent, so each sampled row is exact).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests.gpu_util import (check_layer, check_routing, run_forward, sample_rows, to_dev)
+from workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU machines too
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import mixture_experts_ffn_rmsnorm_b200 as moe  # noqa: E402
+
+_CACHE = {}
+
+
+def setup(name, T=None, max_tokens=None):
+    key = (name, T, max_tokens)
+    if key not in _CACHE:
+        inp = make_inputs(WORKLOADS[name], T=T)
+        layer = moe.MoELayer.from_inputs(inp, max_tokens=max_tokens or inp.shape.T)
+        _CACHE[key] = (inp, layer, oracle.Oracle(inp))
+    return _CACHE[key]
+
+
+def teardown_module(module):
+    for _, layer, _ in _CACHE.values():
+        layer.close()
+    _CACHE.clear()
+
+
+# ------------------------------------------------------------ tiny, full ---
+
+@pytest.mark.parametrize("path", [moe.PATH_PREFILL, moe.PATH_DECODE])
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
+def test_tiny_small_T_both_paths(T, path):
+    inp, layer, orc = setup("tiny", max_tokens=16)
+    h = inp.hidden[:T]
+    out, res, idx, w = run_forward(layer, h, path)
+    assert np.array_equal(res, h)                        # residual <- pre-layer hidden
+    flips = check_routing(orc, h, idx, w)
+    check_layer(orc, h, out, idx, np.arange(T))
+    assert layer.device_status() == 0
+    print(f"T={T} path={path} flips={flips}")
+
+
+def test_tiny_full_prefill():
+    inp, layer, orc = setup("tiny")
+    out, res, idx, w = run_forward(layer, inp.hidden, moe.PATH_AUTO)
+    check_routing(orc, inp.hidden, idx, w)
+    check_layer(orc, inp.hidden, out, idx, np.arange(16))
+
+
+@pytest.mark.parametrize("T", [17, 128, 129, 300, 513])
+def test_ragged_token_counts_span_tiles(T):
+    # several 128-row tiles with a ragged tail, expert groups of every size
+    inp, layer, orc = setup("tiny", T=513, max_tokens=513)
+    h = inp.hidden[:T]
+    out, res, idx, w = run_forward(layer, h, moe.PATH_PREFILL)
+    assert np.array_equal(res, h)
+    check_routing(orc, h, idx, w)
+    check_layer(orc, h, out, idx, np.arange(T))
+
+
+def test_residual_input_is_ignored_and_output_deterministic():
+    inp, layer, orc = setup("tiny")
+    a = run_forward(layer, inp.hidden, moe.PATH_PREFILL, residual_bits=inp.residual)
+    b = run_forward(layer, inp.hidden, moe.PATH_PREFILL)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[2], b[2])
+    c = run_forward(layer, inp.hidden[:4], moe.PATH_DECODE, residual_bits=inp.residual[:4])
+    d = run_forward(layer, inp.hidden[:4], moe.PATH_DECODE)
+    assert np.array_equal(c[0], d[0])
+
+
+# ------------------------------------------------------- full-size configs ---
+
+@pytest.mark.parametrize("T", [1, 2, 4, 8])
+@pytest.mark.parametrize("path", [moe.PATH_DECODE, moe.PATH_PREFILL])
+def test_decode_workload(T, path):
+    inp, layer, orc = setup("decode", T=8, max_tokens=8)
+    h = inp.hidden[:T]
+    out, res, idx, w = run_forward(layer, h, path)
+    assert np.array_equal(res, h)
+    flips = check_routing(orc, h, idx, w)
+    err, bound = check_layer(orc, h, out, idx, np.arange(T))
+    print(f"decode T={T} path={path}: err {err:.3g} bound {bound:.3g} flips {flips}")
+
+
+def test_prefill_workload():
+    inp, layer, orc = setup("prefill")
+    out, res, idx, w = run_forward(layer, inp.hidden, moe.PATH_AUTO)
+    assert np.array_equal(res, inp.hidden)
+    rows = sample_rows(inp.shape.T, 40)
+    flips = check_routing(orc, inp.hidden, idx, w, rows)
+    err, bound = check_layer(orc, inp.hidden, out, idx, rows)
+    print(f"prefill: err {err:.3g} bound {bound:.3g} flips {flips}/{len(rows)}")
+
+
+def test_latent_workload():
+    inp, layer, orc = setup("latent")
+    out, res, idx, w = run_forward(layer, inp.hidden, moe.PATH_AUTO)
+    assert np.array_equal(res, inp.hidden)
+    rows = sample_rows(inp.shape.T, 24)
+    flips = check_routing(orc, inp.hidden, idx, w, rows)
+    err, bound = check_layer(orc, inp.hidden, out, idx, rows)
+    print(f"latent: err {err:.3g} bound {bound:.3g} flips {flips}/{len(rows)}")
+
+
+def test_full_routing_of_prefill_workload_within_tie_window():
+    # every token's routing set (cheap: gate only) against the oracle
+    inp, layer, orc = setup("prefill")
+    T, k = inp.shape.T, inp.shape.k
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    layer.route(to_dev(inp.hidden), idx, w)
+    torch.cuda.synchronize()
+    flips = check_routing(orc, inp.hidden, idx.cpu().numpy(), w.cpu().numpy())
+    print(f"routing flips inside the 1e-5 window: {flips}/{T}")
+
+
+# ------------------------------------------------------------------- sort ---
+
+@pytest.mark.parametrize("name,T,skew", [("tiny", 16, False), ("prefill", 1024, False),
+                                         ("prefill", 1024, True), ("latent", 4096, False)])
+def test_sort_bit_exact(name, T, skew):
+    inp, layer, orc = setup(name)
+    s = inp.shape
+    rng = np.random.default_rng(T)
+    if skew:   # one expert in every token, the rest spread: groups of all sizes
+        idx = np.stack([np.concatenate([[3], rng.choice(np.delete(np.arange(s.E), 3), s.k - 1,
+                                                        replace=False)]) for _ in range(T)])
+    else:
+        idx = np.stack([rng.choice(s.E, s.k, replace=False) for _ in range(T)])
+    idx = idx.astype(np.int32)
+    perm_o, inv_o, off_o = oracle.sort(idx, s.E)
+    R = T * s.k
+    d_idx = torch.from_numpy(idx).cuda()
+    perm = torch.empty(R, dtype=torch.int32, device="cuda")
+    inv = torch.empty(R, dtype=torch.int32, device="cuda")
+    off = torch.empty(s.E + 1, dtype=torch.int32, device="cuda")
+    layer.sort(d_idx, perm, inv, off)
+    torch.cuda.synchronize()
+    assert np.array_equal(perm.cpu().numpy(), perm_o)
+    assert np.array_equal(inv.cpu().numpy(), inv_o)
+    assert np.array_equal(off.cpu().numpy(), off_o)
+
+
+# --------------------------------------------------------- API behaviour ---
+
+def test_graph_capture_and_replay():
+    # no host sync, allocation or D2H inside the forward: it captures
+    inp, layer, orc = setup("tiny")
+    ref = run_forward(layer, inp.hidden, moe.PATH_PREFILL)[0]
+    hid = to_dev(inp.hidden)
+    res = torch.empty_like(hid)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        layer.forward(hid, res, path=moe.PATH_PREFILL, stream=s)
+    hid.copy_(to_dev(inp.hidden))
+    g.replay()
+    torch.cuda.synchronize()
+    from workloads import bf16_to_f32
+    assert np.array_equal(bf16_to_f32(hid.cpu().numpy().view(np.uint16)), ref)
+
+
+def test_host_buffer_entry_point():
+    inp, layer, orc = setup("tiny")
+    ref, ref_res, _, _ = run_forward(layer, inp.hidden, moe.PATH_AUTO)
+    h = torch.from_numpy(inp.hidden.view(np.int16).copy()).pin_memory()
+    r = torch.empty_like(h).pin_memory()
+    layer.forward_host(h, r)
+    torch.cuda.synchronize()
+    from workloads import bf16_to_f32
+    assert np.array_equal(bf16_to_f32(h.numpy().view(np.uint16)), ref)
+    assert np.array_equal(r.numpy().view(np.uint16), inp.hidden)
+
+
+def test_error_codes():
+    inp, layer, orc = setup("tiny")
+    hid = to_dev(inp.hidden)
+    res = torch.empty_like(hid)
+    L = layer.lib
+    assert L.moe_forward(layer.handle, hid.data_ptr(), res.data_ptr(), 0, None) == 4
+    assert L.moe_forward(layer.handle, hid.data_ptr(), res.data_ptr(), 17, None) == 4
+    assert L.moe_forward(layer.handle, None, res.data_ptr(), 4, None) == 2
+    assert L.moe_forward(layer.handle, hid.data_ptr() + 2, res.data_ptr(), 4, None) == 3
+    assert L.moe_forward_path(layer.handle, hid.data_ptr(), res.data_ptr(), 9, 1, None) == 4
+    assert L.moe_forward(None, hid.data_ptr(), res.data_ptr(), 4, None) == 8
+    assert layer.device_status() == 0
+
+
+def test_create_destroy_cycle_and_bad_configs():
+    inp = make_inputs(WORKLOADS["tiny"])
+    for _ in range(3):
+        l2 = moe.MoELayer.from_inputs(inp)
+        l2.close()
+    with pytest.raises(moe.MoEError):
+        moe.MoELayer.from_inputs(make_inputs(WORKLOADS["tiny"].scaled(k=9)))
+    with pytest.raises(moe.MoEError):
+        moe.MoELayer.from_inputs(make_inputs(WORKLOADS["tiny"].scaled(I=100)))
