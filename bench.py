@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of the Nemotron-H MoE FFN layer forward on B200 (tokens/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--tokens T] [--impl ours|reference]
+
+One step = one full forward of the layer (norm, router, top-k, sort, experts,
+shared expert, reduce, residual) over one batch of T synthetic tokens with
+inputs resident in HBM.  The default workload is the decode configuration at
+T=1 (H=2688, E=128, top_k=6, moe_inter=1856, shared 3712, BF16 weights).
+L2 is flushed (256 MB write, then 256 MB read) between timed steps; every step restores the
+same input tokens, so routing and work are identical across steps.
+
+Multi-GPU (torchrun, one rank per GPU): tokens are independent, so every
+rank runs its own replica on its own batch with no data-path collective
+(weak scaling); NCCL is used only for the barrier and the max-over-ranks
+time.  Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle on the host cores instead, on
+a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec"
+UNIT = "tokens/s"
+DEFAULT_TOKENS = {"tiny": 16, "decode": 1, "prefill": 1024, "latent": 4096, "skew_fp8": 8192}
+
+
+# ------------------------------------------------------------------ peaks ---
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------- work per kernel ---
+
+def stage_model(s, T, path, U):
+    """Algorithmic bytes / flops of every kernel the chosen path launches.
+
+    U = distinct routed experts of the step (weights touched once each).
+    Weight bytes use the storage width (2 for BF16, 1 for FP8 + scales).
+    Returns a list of (name, bytes, flops) in launch order.
+    """
+    H, E, k, I, S, L = s.H, s.E, s.k, s.I, s.S, s.L
+    D = s.D
+    R = T * k
+    wb = 1 if s.expert_fp8 else 2
+    up_w = U * I * D * wb + (U * I * 4 if s.expert_fp8 else 0)
+    down_w = U * D * I * wb + (U * D * 4 if s.expert_fp8 else 0)
+    if path == "decode":
+        return [
+            ("decode_route", (E + S) * H * 2 + 3 * T * H * 2 + T * S * 2 + T * E * 4,
+             2 * T * H * (E + S)),
+            ("decode_up_sdown", up_w + H * S * 2 + R * I * 2 + T * H * 4, 2 * R * D * I + 2 * T * S * H),
+            ("decode_down_combine", down_w + T * H * (2 + 4 + 2), 2 * R * I * D),
+        ]
+    st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2, 0)]
+    if L:
+        st.append(("router_gemm_topk+fc1", E * H * 2 + T * 2 * H * 2 + L * H * 2 + T * L * 2,
+                   2 * T * E * H + 2 * T * H * L))
+    else:
+        st.append(("router_gemm_topk", E * H * 2 + T * 2 * H * 2 + R * 8, 2 * T * E * H))
+    st += [
+        ("sort", R * 4 * 3 + (E + 1) * 4, 0),
+        ("gather", 2 * R * D * 2, 0),
+        ("grouped_up_gemm", up_w + S * H * 2 + R * D * 2 + T * H * 2 + R * I * 2 + T * S * 2,
+         2 * R * D * I + 2 * T * H * S),
+        ("grouped_down_gemm", down_w + H * S * 2 + R * I * 2 + T * S * 2 + R * D * 2 + T * H * 4,
+         2 * R * I * D + 2 * T * S * H),
+    ]
+    if L:
+        st += [("latent_reduce", R * L * 2 + T * L * 2, 0),
+               ("fc2_gemm_blend", H * L * 2 + T * L * 2 + T * H * (4 + 2 + 2), 2 * T * L * H)]
+    else:
+        st.append(("combine", R * D * 2 + T * H * 4 + T * H * 2 * 2, 0))
+    return st
+
+
+def roofline_of(name, nbytes, flops, ms, peaks, expert_fp8):
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    tf = peaks["bf16_tflops"] * (2.0 if expert_fp8 and "gemm" in name else 1.0)
+    t_tc = flops / (tf * 1e12) if flops else 0.0
+    if t_tc > t_hbm:
+        ach = flops / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": tf, "unit": "TFLOP/s",
+                "frac": round(ach / tf, 4)}
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm_gbs"], 4)}
+
+
+def kernel_traffic(name):
+    """dram bytes per launch from the committed ncu summary, or None when the
+    kernel's source has changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = d.get("kernels", {}).get(name)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return rec["dram_bytes_per_launch"] if h == rec.get("source_sha256_16") else None
+
+
+# --------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, interval=0.002):
+        self.samples = []
+        self.reasons = 0
+        self.interval = interval
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable"}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples), "source": "nvml in-process"}
+
+
+# --------------------------------------------------------- CPU baseline ---
+
+def cpu_baseline(inp, T, target_s=10.0):
+    """The float64 oracle as it stands, on host threads, over a bounded
+    sample of the same workload (same weights, more tokens)."""
+    import oracle
+    s = inp.shape
+    threads = oracle.default_threads()
+    orc = oracle.Oracle(inp)
+    probe = make_inputs(s, T=max(threads, 1), experts=False).hidden
+    t0 = time.perf_counter()
+    orc.forward(probe, nthreads=threads)
+    per_tok = (time.perf_counter() - t0) / probe.shape[0]
+    n = int(min(4096, max(threads, target_s / max(per_tok, 1e-9))))
+    n = max(threads, (n // threads) * threads)
+    sample = make_inputs(s, T=n, experts=False).hidden
+    t0 = time.perf_counter()
+    orc.forward(sample, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": round(n / dt, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} tokens of the {s.name} workload (same weights), float64 C++ oracle "
+                      f"threaded over tokens, {dt:.1f} s"}
+
+
+# ------------------------------------------------------------ reference ---
+
+def run_reference(args, shape, T, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    inp = make_inputs(shape, T=T)
+    orc = oracle.Oracle(inp)
+    threads = oracle.default_threads()
+    # per-step sample: as many of the T tokens as keep the whole run short
+    t0 = time.perf_counter()
+    orc.forward(inp.hidden[:1], nthreads=threads)
+    per_tok = time.perf_counter() - t0
+    budget = 150.0
+    n = int(max(1, min(T, budget / max(per_tok * (args.steps + args.warmup), 1e-9) * threads)))
+    h = inp.hidden[:n]
+    for _ in range(args.warmup):
+        orc.forward(h, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.forward(h, nthreads=threads)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(shape, T, "oracle"),
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"{n} of the {T} tokens per step, float64 C++ oracle, "
+                                       f"{threads} threads"},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(s, T, path):
+    w = "FP8 E4M3 experts" if s.expert_fp8 else "BF16"
+    lat = f", latent={s.L}" if s.L else ""
+    return {"workload": f"{s.name} T={T} (H={s.H}, E={s.E}, top_k={s.k}, moe_inter={s.I}, "
+                        f"shared={s.S}{lat}, {w}, rsf={s.rsf})",
+            "tokens_per_step": T, "path": path, "l2": "flushed between timed steps (256 MB write + 256 MB read)"}
+
+
+# ------------------------------------------------------------------ ours ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    shape = WORKLOADS[args.workload]
+    T = args.tokens or DEFAULT_TOKENS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, shape, T, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_ffn_rmsnorm_b200 as moe
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    inp = make_inputs(shape, T=T)
+    layer = moe.MoELayer.from_inputs(inp, max_tokens=T)
+    path = "decode" if T <= 8 and shape.L == 0 and not shape.expert_fp8 else "prefill"
+    pristine = torch.from_numpy(inp.hidden.view(np.int16).copy()).cuda()
+    hid = torch.empty_like(pristine)
+    res = torch.empty_like(pristine)
+    flush_w = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_out = torch.empty((), dtype=torch.float32, device="cuda")
+
+    def flush_l2():
+        # write 256 MB (evicts everything), then read another 256 MB so L2
+        # holds clean lines and the next step pays no write-backs
+        flush_w.zero_()
+        torch.amax(flush_r, dim=0, out=flush_out)
+    stream = torch.cuda.current_stream()
+
+    # one untimed step to learn the launch count and the routing
+    hid.copy_(pristine)
+    layer.forward(hid, res)
+    torch.cuda.synchronize()
+    nl = layer.last_launch_count()
+    idx = torch.empty((T, shape.k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, shape.k), dtype=torch.float32, device="cuda")
+    layer.copy_routing(idx, wts)
+    U = int(torch.unique(idx).numel())
+
+    def make_events(n):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in ev:
+            e.record(stream)
+        return ev
+
+    for _ in range(args.warmup):
+        flush_l2()
+        hid.copy_(pristine)
+        layer.forward(hid, res)
+    torch.cuda.synchronize()
+
+    events = [make_events(nl + 1) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush_l2()
+            hid.copy_(pristine)
+            layer.set_stage_events(events[i])
+            layer.forward(hid, res)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+    layer.set_stage_events(None)
+    stage_ms = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(nl)] for ev in events])
+    step_ms = stage_ms.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * T * args.steps / (total_ms * 1e-3)
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    h_host = torch.from_numpy(inp.hidden.view(np.int16).copy()).pin_memory()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    src = inp.hidden.view(np.int16)
+    for i in range(args.steps):
+        h_host.numpy()[...] = src
+        flush_l2()
+        e0[i].record(stream)
+        layer.forward_host(h_host)
+        e1[i].record(stream)
+        stream.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = world * T * args.steps / (e2e_ms * 1e-3)
+
+    peaks = measured_peaks()
+    model = stage_model(shape, T, path, U)
+    mean_stage = stage_ms.mean(axis=0)
+    stages = []
+    for (name, nb, fl), ms in zip(model, mean_stage):
+        r = roofline_of(name, nb, fl, float(ms), peaks, shape.expert_fp8)
+        stages.append({"kernel": name, "ms": round(float(ms), 5),
+                       "share": round(float(ms / mean_stage.sum()), 4), **r})
+    dom = max(stages, key=lambda d: d["ms"])
+    nb = dict((m[0], m) for m in model)[dom["kernel"]]
+    roof = {k: dom[k] for k in ("bound", "achieved", "peak", "unit", "frac")}
+    roof["kernel"] = dom["kernel"]
+    roof["algorithmic"] = nb[1] if dom["bound"] == "hbm" else nb[2]
+    roof["peak_source"] = peaks["source"] + (" (burst copy)" if dom["bound"] == "hbm"
+                                             else " bf16 burst")
+    roof["traffic"] = kernel_traffic(dom["kernel"])
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8+bf16" if shape.expert_fp8 else "bf16", "data": "synthetic",
+            "config": {**config_of(shape, T, path), "global_batch": world * T,
+                       "parallelism": f"replicas x{world}", "distinct_experts": U},
+            "clocks": clk.summary(),
+            "e2e": {"value": round(e2e, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
+            "gpu_launches": nl * args.steps,
+            "roofline": roof,
+            "stages": stages,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inp, T)
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

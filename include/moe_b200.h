@@ -187,6 +187,13 @@ MOE_API moe_status moe_copy_routing(moe_handle* h, int32_t* idx, float* w, int32
  * clear it.  Synchronises the stream (debug use only). */
 MOE_API moe_status moe_get_device_status(moe_handle* h, int32_t* status, void* stream);
 
+/* Profiling: every following moe_forward* call records caller-owned CUDA
+ * events (cudaEvent_t values passed as void*) on its stream: events[0] before
+ * its first kernel launch and events[i] after its i-th launch, for i < count.
+ * The array is borrowed and must stay valid while enabled; count = 0
+ * disables.  Recording adds no device work besides the event records. */
+MOE_API moe_status moe_set_stage_events(moe_handle* h, void* const* events, int32_t count);
+
 /* Number of kernel launches the last moe_forward* call enqueued. */
 MOE_API int32_t moe_last_launch_count(const moe_handle* h);
 

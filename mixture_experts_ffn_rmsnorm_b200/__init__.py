@@ -26,7 +26,8 @@ WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
 
 EXPORTED_SYMBOLS = ("moe_create", "moe_forward", "moe_forward_path", "moe_forward_host",
                     "moe_destroy", "moe_status_string", "moe_route", "moe_sort",
-                    "moe_get_device_status", "moe_last_launch_count", "moe_copy_routing")
+                    "moe_get_device_status", "moe_last_launch_count", "moe_copy_routing",
+                    "moe_set_stage_events")
 
 
 class MoEError(RuntimeError):
@@ -75,6 +76,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_get_device_status": ([V, V, V], ctypes.c_int),
         "moe_last_launch_count": ([V], I32),
         "moe_copy_routing": ([V, V, V, I32, V], ctypes.c_int),
+        "moe_set_stage_events": ([V, V, I32], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -156,6 +158,19 @@ class MoELayer:
         self._check(self.lib.moe_get_device_status(self.handle, ctypes.byref(v),
                                                    _stream_ptr(stream)), "moe_get_device_status")
         return int(v.value)
+
+    def set_stage_events(self, events):
+        """Record torch.cuda.Event objects around each kernel of later forwards
+        (events[0] before the first launch, events[i] after the i-th); None
+        disables.  The events must already exist (recorded once)."""
+        if not events:
+            self._events = None
+            self._check(self.lib.moe_set_stage_events(self.handle, None, 0), "moe_set_stage_events")
+            return
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        self._events = (arr, list(events))
+        self._check(self.lib.moe_set_stage_events(self.handle, arr, len(events)),
+                    "moe_set_stage_events")
 
     def last_launch_count(self) -> int:
         return int(self.lib.moe_last_launch_count(self.handle))

@@ -76,6 +76,8 @@ struct moe_handle {
   bool fp8;
   int gate_bn;     // router GEMM tile width (>= E)
   int last_launches;
+  void* const* stage_events;  // profiling: caller-owned cudaEvent_t array
+  int n_stage_events;
   int last_tokens;    // num_tokens of the last forward
   bool last_decode;   // whether it took the decode path
   // workspace
@@ -240,11 +242,11 @@ moe::GemmClass dense_class(int K, int N, int rows, int epi, void* out, int ldo, 
 
 // Norm + router GEMM with fused top-k (+ fc1 for LatentMoE).
 moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int T,
-                         bool with_fc1, cudaStream_t st, int* launches) {
+                         bool with_fc1, cudaStream_t st, moe::LaunchLog* log) {
   const moe_config& c = h->cfg;
   MOE_TRY(moe::launch_rmsnorm(hidden, static_cast<const bf16*>(h->w.norm_w), residual, h->gate_a,
                               T, c.hidden_size, c.rms_eps, st));
-  ++*launches;
+  log->done(st);
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.tmA[0] = h->tm_gate_a;
@@ -271,25 +273,25 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
   int W = p.cls[0].mtiles + (p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0);
   const int grid = W < h->num_sms ? W : h->num_sms;
   MOE_TRY(moe::launch_grouped_gemm(p, h->gate_bn, false, grid, st));
-  ++*launches;
+  log->done(st);
   return MOE_OK;
 }
 
 moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, cudaStream_t st,
-                           int* launches) {
+                           moe::LaunchLog* log) {
   const moe_config& c = h->cfg;
   const int H = c.hidden_size, k = c.top_k, E = c.num_experts, I = c.moe_inter,
             S = c.shared_inter, L = c.latent_size, D = h->D, R = T * k;
-  moe_status rs = enqueue_route(h, hidden, residual, T, true, st, launches);
+  moe_status rs = enqueue_route(h, hidden, residual, T, true, st, log);
   if (rs != MOE_OK) return rs;
   MOE_TRY(moe::launch_sort(h->idx, T, k, E, h->perm, h->inv, h->off, h->tiles, h->n_mtiles,
                            h->status, st));
-  ++*launches;
+  log->done(st);
   if (L)
     MOE_TRY(moe::launch_gather(h->z, L, h->perm, k, R, D, h->xs, st));
   else
     MOE_TRY(moe::launch_gather(h->gate_a, 2 * H, h->perm, k, R, D, h->xs, st));
-  ++*launches;
+  log->done(st);
 
   // grouped up (+ relu^2): routed class 0 via the tile table, shared class 1
   GemmParams p;
@@ -306,7 +308,7 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.group_off = h->off;
   p.status = h->status;
   MOE_TRY(moe::launch_grouped_gemm(p, 128, false, h->num_sms, st));
-  ++*launches;
+  log->done(st);
 
   // grouped down: routed -> y (bf16, sorted rows), shared -> s (f32)
   p.tmA[0] = h->tm_down_a;
@@ -316,15 +318,15 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.tmB[1] = h->tm_sdown_b;
   p.cls[1] = dense_class(S, H, T, moe::EPI_F32, h->s, H, 128);
   MOE_TRY(moe::launch_grouped_gemm(p, 128, false, h->num_sms, st));
-  ++*launches;
+  log->done(st);
 
   if (!L) {
     MOE_TRY(moe::launch_combine(h->y, h->inv, h->wts, h->s, residual, hidden, T, k, H, st));
-    ++*launches;
+    log->done(st);
     return MOE_OK;
   }
   MOE_TRY(moe::launch_latent_reduce(h->y, h->inv, h->wts, h->m, T, k, L, st));
-  ++*launches;
+  log->done(st);
   GemmParams q;
   std::memset(&q, 0, sizeof(q));
   q.tmA[0] = h->tm_fc2_a;
@@ -336,7 +338,7 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   q.status = h->status;
   const int W = q.cls[0].mtiles * q.cls[0].ntiles;
   MOE_TRY(moe::launch_grouped_gemm(q, 128, false, W < h->num_sms ? W : h->num_sms, st));
-  ++*launches;
+  log->done(st);
   return MOE_OK;
 }
 
@@ -435,7 +437,10 @@ moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t
   if (path == MOE_PATH_DECODE && num_tokens > MOE_DECODE_MAX_TOKENS)
     return MOE_ERR_TOKENS_OUT_OF_RANGE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int launches = 0;
+  moe::LaunchLog log;
+  log.events = h->stage_events;
+  log.nevents = h->n_stage_events;
+  log.begin(s);
   const bool decode = path == MOE_PATH_DECODE ||
                       (path == MOE_PATH_AUTO && num_tokens <= MOE_DECODE_MAX_TOKENS &&
                        moe::decode_supported(h->cfg));
@@ -445,13 +450,14 @@ moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t
     a.w = &h->w;
     a.ws = &h->dec;
     a.status = h->status;
+    a.num_sms = h->num_sms;
     st = moe::enqueue_decode(a, static_cast<bf16*>(hidden), static_cast<bf16*>(residual),
-                             num_tokens, s, &launches);
+                             num_tokens, s, &log);
   } else {
     st = enqueue_prefill(h, static_cast<bf16*>(hidden), static_cast<bf16*>(residual), num_tokens,
-                         s, &launches);
+                         s, &log);
   }
-  h->last_launches = launches;
+  h->last_launches = log.count;
   h->last_tokens = num_tokens;
   h->last_decode = decode;
   return st;
@@ -487,14 +493,14 @@ moe_status moe_route(moe_handle* h, const void* hidden, int32_t num_tokens, int3
   if (!aligned16(hidden)) return MOE_ERR_MISALIGNED;
   if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int launches = 0;
+  moe::LaunchLog log;
   st = enqueue_route(h, static_cast<const bf16*>(hidden), h->stage_r, num_tokens, false, s,
-                     &launches);
+                     &log);
   if (st != MOE_OK) return st;
   const size_t n = size_t(num_tokens) * h->cfg.top_k;
   MOE_TRY(cudaMemcpyAsync(idx, h->idx, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
   MOE_TRY(cudaMemcpyAsync(w, h->wts, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
-  h->last_launches = launches;
+  h->last_launches = log.count;
   return MOE_OK;
 }
 
@@ -533,6 +539,15 @@ moe_status moe_get_device_status(moe_handle* h, int32_t* status, void* stream) {
   MOE_TRY(cudaMemcpyAsync(status, h->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
   MOE_TRY(cudaMemsetAsync(h->status, 0, sizeof(int32_t), s));
   MOE_TRY(cudaStreamSynchronize(s));
+  return MOE_OK;
+}
+
+moe_status moe_set_stage_events(moe_handle* h, void* const* events, int32_t count) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  if (count < 0 || (count > 0 && !events)) return MOE_ERR_NULL_POINTER;
+  h->stage_events = count > 0 ? events : nullptr;
+  h->n_stage_events = count;
   return MOE_OK;
 }
 

@@ -21,6 +21,22 @@ enum EpiKind : int {
   EPI_BLEND = 4,       // out = bf16(acc + blend_s + blend_res)  (LatentMoE fc2)
 };
 
+// Counts the kernels a call enqueues and, when profiling is enabled, records
+// caller-owned CUDA events around them: events[0] before the first launch,
+// events[i] after the i-th.
+struct LaunchLog {
+  int count = 0;
+  void* const* events = nullptr;
+  int nevents = 0;
+  void begin(cudaStream_t s) const {
+    if (nevents > 0) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s);
+  }
+  void done(cudaStream_t s) {
+    ++count;
+    if (count < nevents) cudaEventRecord(static_cast<cudaEvent_t>(events[count]), s);
+  }
+};
+
 // One class of GEMM tiles inside a launch.  A is [rows, K] (K contiguous),
 // B is [groups * N, K]; a tile multiplies 128 rows of A by BN rows of one
 // group of B.

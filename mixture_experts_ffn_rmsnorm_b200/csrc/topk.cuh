@@ -65,4 +65,64 @@ struct TopK {
   }
 };
 
+// Warp-cooperative top-k of one token's E <= 256 logits (same selection rule
+// and weight formula as TopK): lane l owns experts l, l + 32, ...; k rounds
+// of a warp arg-max on (key descending, expert index ascending).  idx[0..k)
+// and w[0..k) are written by the warp (global or shared memory).
+__device__ __forceinline__ void warp_topk(const float* logits, const float* bias, int E, int k,
+                                          float rsf, int* idx, float* w) {
+  const int lane = threadIdx.x & 31;
+  float key[8], sc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    if (e < E) {
+      const float s = 1.0f / (1.0f + expf(-__ldcg(logits + e)));
+      sc[j] = s;
+      key[j] = s + (bias ? bias[e] : 0.0f);
+    } else {
+      sc[j] = 0.f;
+      key[j] = -INFINITY;
+    }
+  }
+  float sum = 0.f, mine = 0.f;
+  for (int r = 0; r < k; ++r) {
+    float bk = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (key[j] > bk) {
+        bk = key[j];
+        be = lane + 32 * j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    float s = 0.f;
+    if ((be & 31) == lane) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (lane + 32 * j == be) {
+          s = sc[j];
+          key[j] = -INFINITY;
+        }
+      }
+    }
+    s = __shfl_sync(0xffffffffu, s, be & 31);
+    sum += s;
+    if (lane == r) {
+      mine = s;
+      idx[r] = be;
+    }
+  }
+  if (lane < k) w[lane] = mine * (rsf / sum);
+}
+
 }  // namespace moe

@@ -15,8 +15,8 @@ Every weight is stored ``[out, in]`` (row-major, ``in`` contiguous).
 
 Streams: the workload seed is split (numpy SeedSequence.spawn) into one
 independent PCG64 stream per array, in this fixed order: norm_w, gate_w,
-gate_bias, up (expert-major), down (expert-major), shared_up, shared_down,
-fc1, fc2, hidden, residual.  Any array can therefore be drawn without the
+gate_bias, up, down, shared_up, shared_down, fc1, fc2, hidden, residual; the
+up and down streams are split once more, one child per expert.  Any array can therefore be drawn without the
 others, and a smaller token count gives a prefix of a larger one.
 """
 from __future__ import annotations
@@ -104,6 +104,12 @@ def skew_alpha() -> float:
 def bf16_bits(a: np.ndarray) -> np.ndarray:
     """float32 -> BF16 bit pattern (uint16), round to nearest even."""
     a = np.ascontiguousarray(a, dtype=np.float32)
+    if a.size >= (1 << 16):
+        try:  # torch's CPU cast is the same RNE rounding, multi-threaded
+            import torch
+            return torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        except ImportError:
+            pass
     u = a.view(np.uint32)
     r = (u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) >> np.uint32(16)
     return r.astype(np.uint16)
@@ -180,18 +186,24 @@ def _normal(rng, shape, std):
     return x
 
 
-def _expert_stack(rng, E, rows, cols, fp8):
-    """E matrices [rows, cols] ~ N(0, 1/cols), drawn expert by expert."""
+def _expert_stack(seq, E, rows, cols, fp8):
+    """E matrices [rows, cols] ~ N(0, 1/cols); expert e draws from child e of
+    the array's seed sequence, so experts are generated in parallel threads."""
+    import concurrent.futures as cf
     std = 1.0 / np.sqrt(cols)
-    if not fp8:
-        out = np.empty((E, rows, cols), dtype=np.uint16)
-        for e in range(E):
-            out[e] = bf16_bits(_normal(rng, (rows, cols), std))
-        return out, None
-    out = np.empty((E, rows, cols), dtype=np.uint8)
-    sc = np.empty((E, rows), dtype=np.float32)
-    for e in range(E):
-        out[e], sc[e] = _quantize_rows_e4m3(_normal(rng, (rows, cols), std))
+    kids = seq.spawn(E)
+    out = np.empty((E, rows, cols), dtype=np.uint8 if fp8 else np.uint16)
+    sc = np.empty((E, rows), dtype=np.float32) if fp8 else None
+
+    def one(e):
+        x = _normal(np.random.Generator(np.random.PCG64(kids[e])), (rows, cols), std)
+        if fp8:
+            out[e], sc[e] = _quantize_rows_e4m3(x)
+        else:
+            out[e] = bf16_bits(x)
+
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(one, range(E)))
     return out, sc
 
 
@@ -201,7 +213,8 @@ _STREAMS = ("norm_w", "gate_w", "gate_bias", "up", "down", "shared_up", "shared_
 
 def _streams(seed: int):
     kids = np.random.SeedSequence(seed).spawn(len(_STREAMS))
-    return {n: np.random.Generator(np.random.PCG64(k)) for n, k in zip(_STREAMS, kids)}
+    return ({n: np.random.Generator(np.random.PCG64(k)) for n, k in zip(_STREAMS, kids)},
+            dict(zip(_STREAMS, kids)))
 
 
 def make_inputs(shape: MoEShape, T: Optional[int] = None,
@@ -216,7 +229,7 @@ def make_inputs(shape: MoEShape, T: Optional[int] = None,
     if T is not None:
         shape = shape.with_tokens(T)
     s = shape
-    rng = _streams(s.seed)
+    rng, seqs = _streams(s.seed)
     norm_w = bf16_bits(rng["norm_w"].uniform(0.5, 1.5, size=s.H).astype(np.float32))
     gate_w = bf16_bits(_normal(rng["gate_w"], (s.E, s.H), np.sqrt(s.gate_scale / s.H)))
     if s.bias == "none":
@@ -236,8 +249,8 @@ def make_inputs(shape: MoEShape, T: Optional[int] = None,
     up_w = down_w = up_scale = down_scale = None
     shared_up_w = shared_down_w = fc1_w = fc2_w = None
     if experts:
-        up_w, up_scale = _expert_stack(rng["up"], s.E, s.I, D, s.expert_fp8)
-        down_w, down_scale = _expert_stack(rng["down"], s.E, D, s.I, s.expert_fp8)
+        up_w, up_scale = _expert_stack(seqs["up"], s.E, s.I, D, s.expert_fp8)
+        down_w, down_scale = _expert_stack(seqs["down"], s.E, D, s.I, s.expert_fp8)
         shared_up_w = bf16_bits(_normal(rng["shared_up"], (s.S, s.H), 1.0 / np.sqrt(s.H)))
         shared_down_w = bf16_bits(_normal(rng["shared_down"], (s.H, s.S), 1.0 / np.sqrt(s.S)))
         if s.L > 0:
