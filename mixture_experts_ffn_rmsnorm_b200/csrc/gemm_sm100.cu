@@ -25,18 +25,21 @@
 namespace moe {
 namespace {
 
-template <int BN, int STAGES, bool FP8>
+// A stage holds 128 bytes of K per row for both operand types: 64 BF16 or
+// 128 E4M3 elements; one tcgen05.mma consumes 32 bytes of K (16 BF16 or
+// 32 E4M3), so the smem layout and descriptors are type independent.
+template <int BN, int STAGES>
 struct Traits {
-  static constexpr int kBK = FP8 ? 128 : 64;        // K elements per stage (128 bytes)
   static constexpr int kABytes = kBM * 128;
   static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kUmmaK = FP8 ? 32 : 16;      // K per tcgen05.mma (32 bytes)
-  static constexpr int kKSteps = kBK / kUmmaK;
+  static constexpr int kKSteps = 4;                 // 4 x 32 bytes of K per stage
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kSmem = STAGES * kStageBytes + 1024 + 256;
   static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
 };
+
+__device__ __forceinline__ int stage_k(const GemmClass& C) { return C.fp8 ? 128 : 64; }
 
 struct Tile {
   int c;        // class
@@ -104,10 +107,10 @@ __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int
   if (p.status) atomicOr(p.status, kStatusWaitTimeout);
 }
 
-template <int BN, int STAGES, bool FP8>
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using Tr = Traits<BN, STAGES, FP8>;
+  using Tr = Traits<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* tiles = smem_raw + pad;
@@ -167,7 +170,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int w = blockIdx.x; w < W && ok; w += gridDim.x) {
         const Tile t = decode_tile<BN>(p, w, W0);
         const GemmClass& C = p.cls[t.c];
-        const int nk = (C.K + Tr::kBK - 1) / Tr::kBK;
+        const int bk = stage_k(C);
+        const int nk = (C.K + bk - 1) / bk;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) {
             record_timeout(p, abort);
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = tiles + stage * Tr::kStageBytes;
           uint8_t* sb = sa + Tr::kABytes;
           mbar_arrive_expect_tx(&full[stage], Tr::kStageBytes);
-          const int kx = kb * Tr::kBK;
+          const int kx = kb * bk;
           const int kbx = C.b_kwrap ? (kx % C.b_kwrap) : kx;
           tma_load_2d(sa, &p.tmA[t.c], &full[stage], kx, t.row0);
           tma_load_2d(sb, &p.tmB[t.c], &full[stage], kbx, t.brow);
@@ -208,14 +212,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = FP8 ? make_idesc(kBM, BN, 0, 0) : make_idesc(kBM, BN, 1, 1);
+      const uint32_t idesc_f16 = make_idesc(kBM, BN, 1, 1);  // BF16 x BF16 -> F32
+      const uint32_t idesc_f8 = make_idesc(kBM, BN, 0, 0);   // E4M3 x E4M3 -> F32
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < W && ok; w += gridDim.x, ++it) {
         const Tile t = decode_tile<BN>(p, w, W0);
-        const int nk = (p.cls[t.c].K + Tr::kBK - 1) / Tr::kBK;
+        const bool f8 = p.cls[t.c].fp8 != 0;
+        const int bk = f8 ? 128 : 64;
+        const int nk = (p.cls[t.c].K + bk - 1) / bk;
         const int ab = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[ab], aph ^ 1u, abort)) {
@@ -238,10 +245,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int kk = 0; kk < Tr::kKSteps; ++kk) {
             const uint64_t koff = uint64_t((kk * 32) >> 4);
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            if (FP8)
-              umma_f8(d, ad + koff, bd + koff, idesc, acc);
+            if (f8)
+              umma_f8(d, ad + koff, bd + koff, idesc_f8, acc);
             else
-              umma_f16(d, ad + koff, bd + koff, idesc, acc);
+              umma_f16(d, ad + koff, bd + koff, idesc_f16, acc);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -325,6 +332,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (C.epi == EPI_RELU2_BF16) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = v[j] > 0.f ? v[j] * v[j] : 0.f;
+              if (C.row_amax) {
+                float m = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) m = fmaxf(m, v[j]);
+                atomicMax(C.row_amax + row, __float_as_uint(m));
+              }
             }
             if (C.epi == EPI_F32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(C.out) +
@@ -376,19 +389,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-template <int BN, int STAGES, bool FP8>
+template <int BN, int STAGES>
 cudaError_t launch_impl(const GemmParams& p, int grid, cudaStream_t stream) {
-  using Tr = Traits<BN, STAGES, FP8>;
-  auto kern = grouped_gemm_kernel<BN, STAGES, FP8>;
+  using Tr = Traits<BN, STAGES>;
+  auto kern = grouped_gemm_kernel<BN, STAGES>;
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, kGemmThreads, Tr::kSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <int BN, int STAGES, bool FP8>
+template <int BN, int STAGES>
 cudaError_t prepare_impl() {
-  using Tr = Traits<BN, STAGES, FP8>;
-  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, STAGES, FP8>,
+  using Tr = Traits<BN, STAGES>;
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, STAGES>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::kSmem);
 }
 
@@ -396,22 +409,13 @@ cudaError_t prepare_impl() {
 
 cudaError_t prepare_grouped_gemm() {
   cudaError_t e;
-  if ((e = prepare_impl<128, 6, false>()) != cudaSuccess) return e;
-  if ((e = prepare_impl<128, 6, true>()) != cudaSuccess) return e;
-  if ((e = prepare_impl<256, 4, false>()) != cudaSuccess) return e;
-  return prepare_impl<256, 4, true>();
+  if ((e = prepare_impl<128, 6>()) != cudaSuccess) return e;
+  return prepare_impl<256, 4>();
 }
 
-cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, bool fp8, int grid,
-                                cudaStream_t stream) {
-  if (bn == 128) {
-    return fp8 ? launch_impl<128, 6, true>(p, grid, stream)
-               : launch_impl<128, 6, false>(p, grid, stream);
-  }
-  if (bn == 256) {
-    return fp8 ? launch_impl<256, 4, true>(p, grid, stream)
-               : launch_impl<256, 4, false>(p, grid, stream);
-  }
+cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStream_t stream) {
+  if (bn == 128) return launch_impl<128, 6>(p, grid, stream);
+  if (bn == 256) return launch_impl<256, 4>(p, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -101,6 +101,13 @@ struct moe_handle {
   bf16* m;         // [Tm, L]   latent weighted sum
   bf16* stage_h;   // [Tm, H]   host-path staging
   bf16* stage_r;   // [Tm, H]
+  // FP8 experts: E4M3 activations with one float scale per row
+  uint8_t* nq;       // [Tm, H]   normed tokens
+  float* nq_scale;   // [Tm]
+  float* xs_scale;   // [Rm]      scale of each sorted row (xs holds E4M3 bytes)
+  unsigned* u_amax;  // [Rm]      running row max of relu^2(up) (float bits)
+  uint8_t* uq;       // [Rm, I]   E4M3 relu^2(up)
+  float* u_scale;    // [Rm]
   moe::DecodeWorkspace dec;
   // tensor maps
   CUtensorMap tm_gate_a, tm_gate_b, tm_fc1_a, tm_fc1_b;
@@ -187,6 +194,14 @@ void carve(moe_handle* h, char* base) {
   h->m = L ? cv.take<bf16>(Tm * L) : nullptr;
   h->stage_h = cv.take<bf16>(Tm * H);
   h->stage_r = cv.take<bf16>(Tm * H);
+  if (h->fp8) {
+    h->nq = cv.take<uint8_t>(Tm * H);
+    h->nq_scale = cv.take<float>(Tm);
+    h->xs_scale = cv.take<float>(Rm);
+    h->u_amax = cv.take<unsigned>(Rm);
+    h->uq = cv.take<uint8_t>(Rm * I);
+    h->u_scale = cv.take<float>(Rm);
+  }
   moe::carve_decode(&h->dec, c, [&](size_t bytes) { return cv.take<char>(bytes); });
   h->ws_bytes = cv.off;
 }
@@ -214,7 +229,8 @@ bool build_maps(moe_handle* h) {
   ok &= make_map(&h->tm_sup_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
   ok &= make_map(&h->tm_sup_b, h->w.shared_up_w, false, H, S, H * 2, 128);
   // grouped down: routed A = u [Rm, I], B = down [E*D, I]; shared A = v, B = [H, S]
-  ok &= make_map(&h->tm_down_a, h->u, f8, I, Rm, I * eb, moe::kBM);
+  ok &= make_map(&h->tm_down_a, f8 ? static_cast<const void*>(h->uq) : h->u, f8, I, Rm, I * eb,
+                 moe::kBM);
   ok &= make_map(&h->tm_down_b, h->w.down_w, f8, I, E * D, I * eb, 128);
   ok &= make_map(&h->tm_sdown_a, h->v, false, S, Tm, S * 2, moe::kBM);
   ok &= make_map(&h->tm_sdown_b, h->w.shared_down_w, false, S, H, S * 2, 128);
@@ -245,7 +261,8 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
                          bool with_fc1, cudaStream_t st, moe::LaunchLog* log) {
   const moe_config& c = h->cfg;
   MOE_TRY(moe::launch_rmsnorm(hidden, static_cast<const bf16*>(h->w.norm_w), residual, h->gate_a,
-                              T, c.hidden_size, c.rms_eps, st));
+                              h->fp8 && with_fc1 ? h->nq : nullptr, h->nq_scale, T,
+                              c.hidden_size, c.rms_eps, st));
   log->done(st);
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -272,7 +289,7 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
   p.status = h->status;
   int W = p.cls[0].mtiles + (p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0);
   const int grid = W < h->num_sms ? W : h->num_sms;
-  MOE_TRY(moe::launch_grouped_gemm(p, h->gate_bn, false, grid, st));
+  MOE_TRY(moe::launch_grouped_gemm(p, h->gate_bn, grid, st));
   log->done(st);
   return MOE_OK;
 }
@@ -288,9 +305,14 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
                            h->status, st));
   log->done(st);
   if (L)
-    MOE_TRY(moe::launch_gather(h->z, L, h->perm, k, R, D, h->xs, st));
+    MOE_TRY(moe::launch_gather(h->z, size_t(L) * 2, h->perm, k, R, D * 2, h->xs, nullptr,
+                               nullptr, st));
+  else if (h->fp8)
+    MOE_TRY(moe::launch_gather(h->nq, size_t(H), h->perm, k, R, D, h->xs, h->nq_scale,
+                               h->xs_scale, st));
   else
-    MOE_TRY(moe::launch_gather(h->gate_a, 2 * H, h->perm, k, R, D, h->xs, st));
+    MOE_TRY(moe::launch_gather(h->gate_a, size_t(2 * H) * 2, h->perm, k, R, D * 2, h->xs,
+                               nullptr, nullptr, st));
   log->done(st);
 
   // grouped up (+ relu^2): routed class 0 via the tile table, shared class 1
@@ -299,6 +321,12 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.tmA[0] = h->tm_up_a;
   p.tmB[0] = h->tm_up_b;
   p.cls[0] = dense_class(D, I, 0, moe::EPI_RELU2_BF16, h->u, I, 128);
+  if (h->fp8) {  // W8A8: acc * token scale * weight-row scale, row max for requantisation
+    p.cls[0].fp8 = 1;
+    p.cls[0].row_scale = h->xs_scale;
+    p.cls[0].col_scale = h->w.up_scale;
+    p.cls[0].row_amax = h->u_amax;
+  }
   p.tmA[1] = h->tm_sup_a;
   p.tmB[1] = h->tm_sup_b;
   p.cls[1] = dense_class(H, S, T, moe::EPI_RELU2_BF16, h->v, S, 128);
@@ -307,17 +335,27 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.n_mtiles = h->n_mtiles;
   p.group_off = h->off;
   p.status = h->status;
-  MOE_TRY(moe::launch_grouped_gemm(p, 128, false, h->num_sms, st));
+  MOE_TRY(moe::launch_grouped_gemm(p, 128, h->num_sms, st));
   log->done(st);
+
+  if (h->fp8) {
+    MOE_TRY(moe::launch_quantize_rows(h->u, h->u_amax, h->uq, h->u_scale, R, I, st));
+    log->done(st);
+  }
 
   // grouped down: routed -> y (bf16, sorted rows), shared -> s (f32)
   p.tmA[0] = h->tm_down_a;
   p.tmB[0] = h->tm_down_b;
   p.cls[0] = dense_class(I, D, 0, moe::EPI_BF16, h->y, D, 128);
+  if (h->fp8) {
+    p.cls[0].fp8 = 1;
+    p.cls[0].row_scale = h->u_scale;
+    p.cls[0].col_scale = h->w.down_scale;
+  }
   p.tmA[1] = h->tm_sdown_a;
   p.tmB[1] = h->tm_sdown_b;
   p.cls[1] = dense_class(S, H, T, moe::EPI_F32, h->s, H, 128);
-  MOE_TRY(moe::launch_grouped_gemm(p, 128, false, h->num_sms, st));
+  MOE_TRY(moe::launch_grouped_gemm(p, 128, h->num_sms, st));
   log->done(st);
 
   if (!L) {
@@ -337,7 +375,7 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   q.blend_res = residual;
   q.status = h->status;
   const int W = q.cls[0].mtiles * q.cls[0].ntiles;
-  MOE_TRY(moe::launch_grouped_gemm(q, 128, false, W < h->num_sms ? W : h->num_sms, st));
+  MOE_TRY(moe::launch_grouped_gemm(q, 128, W < h->num_sms ? W : h->num_sms, st));
   log->done(st);
   return MOE_OK;
 }
@@ -386,7 +424,7 @@ moe_status moe_create(const moe_config* config, const moe_weights* weights, moe_
   h->D = config->latent_size ? config->latent_size : config->hidden_size;
   h->fp8 = config->expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE;
   h->gate_bn = config->num_experts <= 128 ? 128 : 256;
-  if (h->fp8) {  // the FP8 grouped GEMMs are not wired yet
+  if (h->fp8 && config->latent_size > 0) {  // FP8 experts are wired for the direct layer
     delete h;
     return MOE_ERR_INVALID_CONFIG;
   }

@@ -52,6 +52,8 @@ struct GemmClass {
   int ldo;                // output row stride in elements
   const float* col_scale; // [groups, N] per-output-column scale (FP8 weights) or null
   const float* row_scale; // [rows] per-A-row scale or null
+  int fp8;                // operands are E4M3 (kind::f8f6f4, 128 K elements per stage)
+  unsigned* row_amax;     // per output row max (float bits, values >= 0) or null
 };
 
 struct GemmParams {
@@ -78,22 +80,30 @@ struct GemmParams {
   int* status;
 };
 
-// Launch the persistent grouped GEMM (bn = 128 or 256; fp8 = E4M3 operands).
-cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, bool fp8, int grid,
-                                cudaStream_t stream);
+// Launch the persistent grouped GEMM (bn = 128 or 256); the operand type is
+// a per-class property (GemmClass::fp8).
+cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStream_t stream);
 // Set the dynamic shared memory limit of every GEMM instantiation on the
 // current device (call once per device before launching).
 cudaError_t prepare_grouped_gemm();
 
 // Routing / sort / data movement kernels (route.cu).
+// normed_q/normed_scale (nullable): per-token E4M3 copy of the normed rows.
 cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* norm_w,
-                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, int T, int H,
-                           float eps, cudaStream_t stream);
+                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, uint8_t* normed_q,
+                           float* normed_scale, int T, int H, float eps, cudaStream_t stream);
 size_t sort_smem_bytes(int E);
 cudaError_t launch_sort(const int* idx, int T, int k, int E, int* perm, int* inv, int* off,
                         int2* tile_table, int* n_mtiles, int* status, cudaStream_t stream);
-cudaError_t launch_gather(const __nv_bfloat16* X, int ldx, const int* perm, int k, int R, int D,
-                          __nv_bfloat16* xs, cudaStream_t stream);
+// Row gather: xs[p] = X[perm[p] / k] (row_bytes per row; ldx_bytes source
+// stride); optionally scales: xs_scale[p] = scale[perm[p] / k].
+cudaError_t launch_gather(const void* X, size_t ldx_bytes, const int* perm, int k, int R,
+                          int row_bytes, void* xs, const float* scale, float* xs_scale,
+                          cudaStream_t stream);
+// Per-row E4M3 quantisation of u [R, I] (bf16) with the row maxima amax
+// (float bits, reset to 0 afterwards): uq = sat(u / s), s = amax / 448.
+cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* amax, uint8_t* uq,
+                                 float* scale, int R, int I, cudaStream_t stream);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* inv, const float* w,
                            const float* s, const __nv_bfloat16* residual,
                            __nv_bfloat16* hidden, int T, int k, int H, cudaStream_t stream);

@@ -2,6 +2,8 @@
 // router input), the stable sort by expert, the row gather feeding the
 // grouped up-GEMM, and the unpermute + weighted reduce fused with the shared
 // expert and the residual add.
+#include <cuda_fp8.h>
+
 #include "moe_internal.h"
 #include "ptx.cuh"
 
@@ -29,15 +31,48 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
 
 constexpr int kNormThreads = 256;
 
+__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, w) : v + w;
+  }
+  __syncthreads();  // red may still be read by the previous reduction
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float x = threadIdx.x < kNormThreads / 32 ? red[threadIdx.x] : 0.f;  // identity of both
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float w = __shfl_xor_sync(0xffffffffu, x, o);
+      x = is_max ? fmaxf(x, w) : x + w;
+    }
+    if (threadIdx.x == 0) red[0] = x;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+// E4M3 bits of x (round to nearest even, saturating to +-448).
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xFFFFu) | (hi << 16);
+}
+
 // RMSNorm of one token per block (NemotronMoeLayer `prefill`: rms_norm_residual
 // writes the normed activations and the residual).  residual <- hidden; the
 // normed vector n = x * rsqrt(mean(x^2) + eps) * w is written as two BF16
 // halves into gate_a [T, 2H]: hi = bf16(n) (this is also the experts' input)
 // and lo = bf16(n - hi), so the router GEMM on [hi | lo] x [G | G] sees n to
 // about 16 significant bits (FP32-accurate logits from BF16 tensor cores).
+// With FP8 experts it also writes an E4M3 copy of n with one float scale per
+// token (scale = max|n| / 448).
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ norm_w,
-    __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ gate_a, int H, float eps) {
+    __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ gate_a,
+    uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale, int H, float eps) {
+  __shared__ float red[kNormThreads / 32];
   const int t = blockIdx.x;
   const uint4* x = reinterpret_cast<const uint4*>(hidden + size_t(t) * H);
   uint4* res = reinterpret_cast<uint4*>(residual + size_t(t) * H);
@@ -51,22 +86,11 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
 #pragma unroll
     for (int j = 0; j < 8; ++j) ss += f[j] * f[j];
   }
-  __shared__ float red[kNormThreads / 32];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < kNormThreads / 32 ? red[threadIdx.x] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (threadIdx.x == 0) red[0] = v;
-  }
-  __syncthreads();
-  const float r = rsqrtf(red[0] / float(H) + eps);
+  const float r = rsqrtf(block_reduce(ss, red, false) / float(H) + eps);
   const uint4* w = reinterpret_cast<const uint4*>(norm_w);
   uint4* hi = reinterpret_cast<uint4*>(gate_a + size_t(t) * 2 * H);
   uint4* lo = hi + nv;
+  float amax = 0.f;
   for (int i = threadIdx.x; i < nv; i += kNormThreads) {
     float f[8], g[8], h[8], l[8];
     unpack8(x[i], f);
@@ -76,9 +100,48 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
       const float n = f[j] * r * g[j];
       h[j] = __bfloat162float(__float2bfloat16_rn(n));
       l[j] = n - h[j];
+      amax = fmaxf(amax, fabsf(n));
     }
     hi[i] = pack8(h);
     lo[i] = pack8(l);
+  }
+  if (!normed_q) return;
+  amax = block_reduce(amax, red, true);
+  const float scale = amax > 0.f ? amax / 448.f : 1.f;
+  const float inv = 1.f / scale;
+  if (threadIdx.x == 0) normed_scale[t] = scale;
+  uint2* q = reinterpret_cast<uint2*>(normed_q + size_t(t) * H);
+  for (int i = threadIdx.x; i < nv; i += kNormThreads) {
+    float f[8], g[8], n[8];
+    unpack8(x[i], f);
+    unpack8(w[i], g);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) n[j] = f[j] * r * g[j] * inv;
+    q[i] = make_uint2(e4m3x4(n[0], n[1], n[2], n[3]), e4m3x4(n[4], n[5], n[6], n[7]));
+  }
+}
+
+// uq[p] = E4M3(u[p] / s_p), s_p = amax_p / 448; amax_p reset to 0 for the
+// next forward.  One block per row.
+__global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ u,
+                                     unsigned* __restrict__ amax, uint8_t* __restrict__ uq,
+                                     float* __restrict__ scale, int I) {
+  const int p = blockIdx.x;
+  const float m = __uint_as_float(amax[p]);
+  const float s = m > 0.f ? m / 448.f : 1.f;
+  const float inv = 1.f / s;
+  const uint4* src = reinterpret_cast<const uint4*>(u + size_t(p) * I);
+  uint2* dst = reinterpret_cast<uint2*>(uq + size_t(p) * I);
+  for (int i = threadIdx.x; i < I / 8; i += blockDim.x) {
+    float f[8];
+    unpack8(src[i], f);
+    dst[i] = make_uint2(e4m3x4(f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv),
+                        e4m3x4(f[4] * inv, f[5] * inv, f[6] * inv, f[7] * inv));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    scale[p] = s;
+    amax[p] = 0u;
   }
 }
 
@@ -164,17 +227,20 @@ __global__ void __launch_bounds__(kSortThreads) sort_kernel(
   }
 }
 
-// xs[p, :] = X[perm[p] / k, :]: one warp per sorted row, 16-byte moves.
-__global__ void gather_kernel(const __nv_bfloat16* __restrict__ X, int ldx,
-                              const int* __restrict__ perm, int k, int R, int D,
-                              __nv_bfloat16* __restrict__ xs) {
+// xs[p, :] = X[perm[p] / k, :] (row_bytes per row): one warp per sorted
+// row, 16-byte moves; with FP8 inputs the token scale travels along.
+__global__ void gather_kernel(const uint8_t* __restrict__ X, size_t ldx,
+                              const int* __restrict__ perm, int k, int R, int row_bytes,
+                              uint8_t* __restrict__ xs, const float* __restrict__ scale,
+                              float* __restrict__ xs_scale) {
   const int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (p >= R) return;
   const int lane = threadIdx.x & 31;
   const int t = perm[p] / k;
   const uint4* src = reinterpret_cast<const uint4*>(X + size_t(t) * ldx);
-  uint4* dst = reinterpret_cast<uint4*>(xs + size_t(p) * D);
-  for (int i = lane; i < D / 8; i += 32) dst[i] = src[i];
+  uint4* dst = reinterpret_cast<uint4*>(xs + size_t(p) * row_bytes);
+  for (int i = lane; i < row_bytes / 16; i += 32) dst[i] = src[i];
+  if (scale && lane == 0) xs_scale[p] = scale[t];
 }
 
 // hidden[t] = bf16(residual[t] + s[t] + sum_j w[t,j] * y[inv[t*k + j]])
@@ -238,9 +304,17 @@ __global__ void latent_reduce_kernel(const __nv_bfloat16* __restrict__ y,
 }  // namespace
 
 cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* norm_w,
-                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, int T, int H,
-                           float eps, cudaStream_t stream) {
-  rmsnorm_kernel<<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, H, eps);
+                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, uint8_t* normed_q,
+                           float* normed_scale, int T, int H, float eps, cudaStream_t stream) {
+  rmsnorm_kernel<<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, normed_q,
+                                                 normed_scale, H, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* amax, uint8_t* uq,
+                                 float* scale, int R, int I, cudaStream_t stream) {
+  if (R <= 0) return cudaSuccess;
+  quantize_rows_kernel<<<R, 128, 0, stream>>>(u, amax, uq, scale, I);
   return cudaGetLastError();
 }
 
@@ -259,10 +333,13 @@ cudaError_t launch_sort(const int* idx, int T, int k, int E, int* perm, int* inv
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const __nv_bfloat16* X, int ldx, const int* perm, int k, int R, int D,
-                          __nv_bfloat16* xs, cudaStream_t stream) {
+cudaError_t launch_gather(const void* X, size_t ldx_bytes, const int* perm, int k, int R,
+                          int row_bytes, void* xs, const float* scale, float* xs_scale,
+                          cudaStream_t stream) {
   const int warps = 8;
-  gather_kernel<<<(R + warps - 1) / warps, warps * 32, 0, stream>>>(X, ldx, perm, k, R, D, xs);
+  gather_kernel<<<(R + warps - 1) / warps, warps * 32, 0, stream>>>(
+      static_cast<const uint8_t*>(X), ldx_bytes, perm, k, R, row_bytes,
+      static_cast<uint8_t*>(xs), scale, xs_scale);
   return cudaGetLastError();
 }
 

@@ -25,10 +25,11 @@ import mixture_experts_ffn_rmsnorm_b200 as moe  # noqa: E402
 _CACHE = {}
 
 
-def setup(name, T=None, max_tokens=None):
-    key = (name, T, max_tokens)
+def setup(name, T=None, max_tokens=None, **over):
+    key = (name, T, max_tokens, tuple(sorted(over.items())))
     if key not in _CACHE:
-        inp = make_inputs(WORKLOADS[name], T=T)
+        shape = WORKLOADS[name].scaled(**over) if over else WORKLOADS[name]
+        inp = make_inputs(shape, T=T)
         layer = moe.MoELayer.from_inputs(inp, max_tokens=max_tokens or inp.shape.T)
         _CACHE[key] = (inp, layer, oracle.Oracle(inp))
     return _CACHE[key]
@@ -115,6 +116,33 @@ def test_latent_workload():
     flips = check_routing(orc, inp.hidden, idx, w, rows)
     err, bound = check_layer(orc, inp.hidden, out, idx, rows)
     print(f"latent: err {err:.3g} bound {bound:.3g} flips {flips}/{len(rows)}")
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 129, 300])
+def test_tiny_fp8_experts(T):
+    # E4M3 experts with per-row scales; activations quantised per row on the GPU
+    inp, layer, orc = setup("tiny", T=300, max_tokens=300, expert_fp8=True)
+    h = inp.hidden[:T]
+    out, res, idx, w = run_forward(layer, h, moe.PATH_AUTO)
+    assert np.array_equal(res, h)
+    check_routing(orc, h, idx, w)
+    err, bound = check_layer(orc, h, out, idx, np.arange(T), expert_fp8=True)
+    print(f"tiny fp8 T={T}: err {err:.3g} bound {bound:.3g}")
+    assert layer.device_status() == 0
+
+
+def test_skewed_fp8_workload():
+    inp, layer, orc = setup("skew_fp8")
+    out, res, idx, w = run_forward(layer, inp.hidden, moe.PATH_AUTO)
+    assert np.array_equal(res, inp.hidden)
+    cnt = np.bincount(idx.reshape(-1), minlength=inp.shape.E)
+    skew = cnt.max() / (inp.shape.T * inp.shape.k / inp.shape.E)
+    assert skew > 10, f"hottest expert only {skew:.1f}x the mean"
+    rows = sample_rows(inp.shape.T, 32)
+    flips = check_routing(orc, inp.hidden, idx, w, rows)
+    err, bound = check_layer(orc, inp.hidden, out, idx, rows, expert_fp8=True)
+    print(f"skew fp8: hottest/mean {skew:.1f} err {err:.3g} bound {bound:.3g} flips {flips}")
+    assert layer.device_status() == 0
 
 
 def test_full_routing_of_prefill_workload_within_tie_window():
