@@ -80,7 +80,7 @@ def stage_model(s, T, path, U):
             ("decode_up_sdown", up_w + H * S * 2 + R * I * 2 + T * H * 4, 2 * R * D * I + 2 * T * S * H),
             ("decode_down_combine", down_w + T * H * (2 + 4 + 2), 2 * R * I * D),
         ]
-    st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2, 0)]
+    st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2 + (T * H if s.expert_fp8 else 0), 0)]
     if L:
         st.append(("router_gemm_topk+fc1", E * H * 2 + T * 2 * H * 2 + L * H * 2 + T * L * 2,
                    2 * T * E * H + 2 * T * H * L))
@@ -88,10 +88,14 @@ def stage_model(s, T, path, U):
         st.append(("router_gemm_topk", E * H * 2 + T * 2 * H * 2 + R * 8, 2 * T * E * H))
     st += [
         ("sort", R * 4 * 3 + (E + 1) * 4, 0),
-        ("gather", 2 * R * D * 2, 0),
-        ("grouped_up_gemm", up_w + S * H * 2 + R * D * 2 + T * H * 2 + R * I * 2 + T * S * 2,
+        ("gather", 2 * R * D * wb, 0),
+        ("grouped_up_gemm", up_w + S * H * 2 + R * D * wb + T * H * 2 + R * I * 2 + T * S * 2,
          2 * R * D * I + 2 * T * H * S),
-        ("grouped_down_gemm", down_w + H * S * 2 + R * I * 2 + T * S * 2 + R * D * 2 + T * H * 4,
+    ]
+    if s.expert_fp8:
+        st.append(("quantize_rows", R * I * 2 + R * I + R * 8, 0))
+    st += [
+        ("grouped_down_gemm", down_w + H * S * 2 + R * I * wb + T * S * 2 + R * D * 2 + T * H * 4,
          2 * R * I * D + 2 * T * S * H),
     ]
     if L:
