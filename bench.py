@@ -75,10 +75,11 @@ def stage_model(s, T, path, U):
     down_w = U * D * I * wb + (U * D * 4 if s.expert_fp8 else 0)
     if path == "decode":
         return [
-            ("decode_route", (E + S) * H * 2 + 3 * T * H * 2 + T * S * 2 + T * E * 4,
-             2 * T * H * (E + S)),
-            ("decode_up_sdown", up_w + H * S * 2 + R * I * 2 + T * H * 4, 2 * R * D * I + 2 * T * S * H),
-            ("decode_down_combine", down_w + T * H * (2 + 4 + 2), 2 * R * I * D),
+            ("decode_route", E * H * 2 + 3 * T * H * 2 + T * E * 4, 2 * T * H * E),
+            ("decode_up_gemm", up_w + S * H * 2 + T * H * 2 + R * I * 2 + T * S * 2,
+             2 * R * D * I + 2 * T * H * S),
+            ("decode_down_gemm", down_w + H * S * 2 + R * I * 2 + T * S * 2 + T * H * 2 * 2,
+             2 * R * I * D + 2 * T * S * H),
         ]
     st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2 + (T * H if s.expert_fp8 else 0), 0)]
     if L:
@@ -276,6 +277,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the forward eagerly each step instead of replaying a CUDA graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -339,7 +342,31 @@ def main():
         layer.forward(hid, res)
     torch.cuda.synchronize()
 
-    events = [make_events(nl + 1) for _ in range(args.steps)]
+    # The step: one replay of a CUDA graph of the forward (what a serving loop
+    # does for a layer), or an eager call with --eager.  A second graph with
+    # CUDA events captured between the kernels gives the per-kernel times.
+    graph = prof_graph = None
+    prof_events = make_events(nl + 1)
+    if not args.eager:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            layer.forward(hid, res, stream=side)
+        prof_graph = torch.cuda.CUDAGraph()
+        layer.set_stage_events(prof_events)
+        with torch.cuda.graph(prof_graph, stream=side):
+            layer.forward(hid, res, stream=side)
+        layer.set_stage_events(None)
+        stream.wait_stream(side)
+        for _ in range(args.warmup):
+            flush_l2()
+            hid.copy_(pristine)
+            graph.replay()
+        torch.cuda.synchronize()
+
+    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -348,21 +375,39 @@ def main():
         for i in range(args.steps):
             flush_l2()
             hid.copy_(pristine)
-            layer.set_stage_events(events[i])
-            layer.forward(hid, res)
+            e_start[i].record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                layer.forward(hid, res)
+            e_end[i].record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-    layer.set_stage_events(None)
-    stage_ms = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(nl)] for ev in events])
-    step_ms = stage_ms.sum(axis=1)
+    step_ms = np.array([a.elapsed_time(b) for a, b in zip(e_start, e_end)])
     total_ms = float(step_ms.sum())
     if world > 1:
         t = torch.tensor([total_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
     value = world * T * args.steps / (total_ms * 1e-3)
+
+    # per-kernel device times: events recorded between the launches
+    n_prof = min(args.steps, 50)
+    stage_ms = np.zeros((n_prof, nl))
+    if prof_graph is None:
+        layer.set_stage_events(prof_events)
+    for i in range(n_prof):
+        flush_l2()
+        hid.copy_(pristine)
+        if prof_graph is not None:
+            prof_graph.replay()
+        else:
+            layer.forward(hid, res)
+        torch.cuda.synchronize()
+        stage_ms[i] = [prof_events[j].elapsed_time(prof_events[j + 1]) for j in range(nl)]
+    layer.set_stage_events(None)
 
     # end to end through the host-buffer entry point (pinned host memory)
     h_host = torch.from_numpy(inp.hidden.view(np.int16).copy()).pin_memory()
@@ -385,6 +430,8 @@ def main():
 
     peaks = measured_peaks()
     model = stage_model(shape, T, path, U)
+    if len(model) != nl:  # keep the JSON honest if the launch list changed
+        model = [(f"kernel_{j}", 0, 0) for j in range(nl)]
     mean_stage = stage_ms.mean(axis=0)
     stages = []
     for (name, nb, fl), ms in zip(model, mean_stage):
@@ -408,7 +455,8 @@ def main():
             "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8+bf16" if shape.expert_fp8 else "bf16", "data": "synthetic",
             "config": {**config_of(shape, T, path), "global_batch": world * T,
-                       "parallelism": f"replicas x{world}", "distinct_experts": U},
+                       "parallelism": f"replicas x{world}", "distinct_experts": U,
+                       "launch": "eager" if graph is None else "cuda_graph_replay"},
             "clocks": clk.summary(),
             "e2e": {"value": round(e2e, 2), "unit": UNIT,
                     "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},

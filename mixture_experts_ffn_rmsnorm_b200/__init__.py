@@ -54,11 +54,15 @@ _lib = None
 
 
 def load_library(path: Optional[str] = None) -> ctypes.CDLL:
-    """Load libmoe_b200.so (building it first if it is absent and nvcc exists)."""
+    """Load libmoe_b200.so (building it first if it is absent and nvcc exists).
+
+    The MOE_B200_LIBRARY environment variable names another build of the same
+    library to load instead (e.g. one compiled with different tile sizes).
+    """
     global _lib
     if _lib is not None:
         return _lib
-    p = path or LIB_PATH
+    p = path or os.environ.get("MOE_B200_LIBRARY") or LIB_PATH
     if not os.path.exists(p):
         from . import build as _build
         _build.build()

@@ -1,8 +1,14 @@
 // Small-batch decode path (1 <= T <= 8): the layer is weight-streaming at
-// these sizes, so it runs as bandwidth-bound GEMVs that read each distinct
-// routed expert's weights once for all tokens routed to it, plus the shared
-// expert's weights once (NemotronMoeLayer `decode`; MoeLayer `forward_k2` /
-// `forward_k3` for the batched small-T idea).
+// these sizes (NemotronMoeLayer `decode`; MoeLayer `forward_k2`/`forward_k3`
+// batch a few tokens through one weight sweep).  Three launches:
+//   decode_route (CUDA cores): RMSNorm, FP32 router logits, sigmoid top-k,
+//       the distinct-expert segment table and the tile lists of the next two
+//       launches.
+//   grouped GEMM, up (tcgen05, weights x tokens, N = 16): relu^2 of every
+//       distinct routed expert's up rows and of the shared expert's.
+//   grouped GEMM, down (split by segment): every segment's down rows; the last
+//       segment of a 128-row tile to finish sums all segments in a fixed order
+//       with the residual into hidden.
 #pragma once
 
 #include <stddef.h>
@@ -14,22 +20,25 @@
 namespace moe {
 
 constexpr int kDecodeMaxT = MOE_DECODE_MAX_TOKENS;
+constexpr int kDecodeN = 16;  // token columns of a decode tile (UMMA N)
 
 struct DecodeWorkspace {
-  __nv_bfloat16* normed;   // [8, H]  bf16(n), the experts' input
+  __nv_bfloat16* x16;      // [16, H]  bf16(n) of the tokens (rows >= T unused)
   float* logits;           // [8, E]
   int* idx;                // [8, k]
   float* w;                // [8, k]
-  int* slot_expert;        // [Umax] distinct routed experts, first-use order
-  int* slot_cnt;           // [Umax] tokens routed to the slot
-  int* slot_tok;           // [Umax, 8] token of the slot's j-th pair
-  int* slot_pair;          // [Umax, 8] flat pair index t*k + j
-  float* slot_w;           // [Umax, 8] routing weight of the pair
-  int* n_slots;            // [1]
+  int* seg_expert;         // [Umax + 1] expert of segment s >= 1 (segment 0 = shared)
+  float* seg_w;            // [Umax + 1, 16] routing weight of token t in segment s (0 = not routed)
+  int* n_segments;         // [1] 1 + distinct experts
   unsigned* counter;       // [1] router blocks finished (self-resetting)
-  __nv_bfloat16* uo;       // [8*k, I] relu^2(up) per (token, slot) pair
-  __nv_bfloat16* vo;       // [8, S]   shared relu^2(up)
-  float* sh;               // [8, H]   shared down output
+  DecodeTile* tiles_up;    // [Umax * ceil(I/128) + ceil(S/128)]
+  int* n_tiles_up;         // [1]
+  DecodeTile* tiles_down;  // [(Umax + 1) * ceil(H/128)]
+  int* n_tiles_down;       // [1]
+  __nv_bfloat16* ub;       // [(Umax + 1) * 16, I] w_t * relu^2(up) per segment, token-major
+  __nv_bfloat16* vb;       // [16, S] shared relu^2(up), token-major
+  float* partial;          // [(Umax + 1), H, 16] down output per segment
+  unsigned* mt_counter;    // [ceil(H/128)] segments finished per row tile (self-resetting)
 };
 
 inline int decode_max_slots(const moe_config& c) {
@@ -37,39 +46,46 @@ inline int decode_max_slots(const moe_config& c) {
   return p < c.num_experts ? p : c.num_experts;
 }
 
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
 template <class Take>
 void carve_decode(DecodeWorkspace* d, const moe_config& c, Take take) {
-  const size_t T = kDecodeMaxT, k = c.top_k, E = c.num_experts, H = c.hidden_size;
+  const size_t k = c.top_k, E = c.num_experts, H = c.hidden_size, I = c.moe_inter,
+               S = c.shared_inter;
   const size_t U = decode_max_slots(c);
-  d->normed = reinterpret_cast<__nv_bfloat16*>(take(T * H * 2));
-  d->logits = reinterpret_cast<float*>(take(T * E * 4));
-  d->idx = reinterpret_cast<int*>(take(T * k * 4));
-  d->w = reinterpret_cast<float*>(take(T * k * 4));
-  d->slot_expert = reinterpret_cast<int*>(take(U * 4));
-  d->slot_cnt = reinterpret_cast<int*>(take(U * 4));
-  d->slot_tok = reinterpret_cast<int*>(take(U * T * 4));
-  d->slot_pair = reinterpret_cast<int*>(take(U * T * 4));
-  d->slot_w = reinterpret_cast<float*>(take(U * T * 4));
-  d->n_slots = reinterpret_cast<int*>(take(4));
+  d->x16 = reinterpret_cast<__nv_bfloat16*>(take(kDecodeN * H * 2));
+  d->logits = reinterpret_cast<float*>(take(kDecodeMaxT * E * 4));
+  d->idx = reinterpret_cast<int*>(take(kDecodeMaxT * k * 4));
+  d->w = reinterpret_cast<float*>(take(kDecodeMaxT * k * 4));
+  d->seg_expert = reinterpret_cast<int*>(take((U + 1) * 4));
+  d->seg_w = reinterpret_cast<float*>(take((U + 1) * kDecodeN * 4));
+  d->n_segments = reinterpret_cast<int*>(take(4));
   d->counter = reinterpret_cast<unsigned*>(take(4));
-  d->uo = reinterpret_cast<__nv_bfloat16*>(take(T * k * c.moe_inter * 2));
-  d->vo = reinterpret_cast<__nv_bfloat16*>(take(T * c.shared_inter * 2));
-  d->sh = reinterpret_cast<float*>(take(T * H * 4));
+  d->tiles_up = reinterpret_cast<DecodeTile*>(
+      take((U * cdiv(int(I), kBM) + cdiv(int(S), kBM)) * sizeof(DecodeTile)));
+  d->n_tiles_up = reinterpret_cast<int*>(take(4));
+  d->tiles_down =
+      reinterpret_cast<DecodeTile*>(take((U + 1) * cdiv(int(H), kBM) * sizeof(DecodeTile)));
+  d->n_tiles_down = reinterpret_cast<int*>(take(4));
+  d->ub = reinterpret_cast<__nv_bfloat16*>(take((U + 1) * kDecodeN * I * 2));
+  d->vb = reinterpret_cast<__nv_bfloat16*>(take(kDecodeN * S * 2));
+  d->partial = reinterpret_cast<float*>(take((U + 1) * H * kDecodeN * 4));
+  d->mt_counter = reinterpret_cast<unsigned*>(take(cdiv(int(H), kBM) * 4));
 }
 
-struct DecodeArgs {
+struct DecodeRouteArgs {
   const moe_config* cfg;
   const moe_weights* w;
   const DecodeWorkspace* ws;
-  int* status;
-  int num_sms;
+  const __nv_bfloat16* hidden;
+  __nv_bfloat16* residual;
+  int T;
 };
 
-// Whether the decode kernels cover this configuration (direct layer with
-// BF16 experts, at most MOE_MAX_EXPERTS experts).
+// Whether the decode path covers this configuration (direct layer, BF16
+// experts, the router rows fit the kernel's shared memory).
 bool decode_supported(const moe_config& c);
 cudaError_t prepare_decode();
-moe_status enqueue_decode(const DecodeArgs& a, __nv_bfloat16* hidden, __nv_bfloat16* residual,
-                          int T, cudaStream_t stream, LaunchLog* log);
+cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t stream);
 
 }  // namespace moe

@@ -34,25 +34,38 @@ struct Traits {
   static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kKSteps = 4;                 // 4 x 32 bytes of K per stage
-  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
   static constexpr int kSmem = STAGES * kStageBytes + 1024 + 256;
-  static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
+  static_assert(kTmemCols == 32 || kTmemCols == 256 || kTmemCols == 512,
+                "TMEM allocation must be a power of two >= 32");
 };
 
 __device__ __forceinline__ int stage_k(const GemmClass& C) { return C.fp8 ? 128 : 64; }
 
 struct Tile {
   int c;        // class
-  int e;        // group (expert) index
-  int row0;     // first A row
-  int row_end;  // first A row not stored
+  int e;        // group (expert) index; decode: segment
+  int row0;     // first A row; decode: first output row inside the segment
+  int row_end;  // first row not stored
   int n0;       // first output column
   int brow;     // first B row
+  int arow;     // first A row to load
 };
 
 template <int BN>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w, int W0) {
   Tile t;
+  if (p.dec_tiles) {
+    const DecodeTile d = p.dec_tiles[w];
+    t.c = d.cls;
+    t.e = d.seg;
+    t.row0 = d.m0;
+    t.row_end = p.dec.M[d.cls];
+    t.n0 = 0;
+    t.brow = d.brow;
+    t.arow = d.arow;
+    return t;
+  }
   if (w < W0) {
     const int nt = p.cls[0].ntiles;
     const int mt = w / nt;
@@ -81,6 +94,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w, int W0) 
     t.n0 = ni * BN;
   }
   t.brow = t.e * p.cls[t.c].N + t.n0;
+  t.arow = t.row0;
   return t;
 }
 
@@ -105,6 +119,70 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
 __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort) {
   *abort = 1;
   if (p.status) atomicOr(p.status, kStatusWaitTimeout);
+}
+
+// Decode epilogues (BN = 16: 128 weight rows x 16 token columns).
+__device__ __forceinline__ void decode_epilogue(const GemmParams& p, const Tile& t, uint32_t tb,
+                                                int rloc, int lane) {
+  __shared__ int last_flag;
+  const DecodeEpilogue& d = p.dec;
+  const GemmClass& C = p.cls[t.c];
+  uint32_t r[16];
+  tmem_ld_32x32b_x16(tb, r);
+  tmem_ld_wait();
+  const int i = t.row0 + rloc;  // output row inside the segment's matrix
+  const int M = d.M[t.c];
+  if (C.epi == EPI_DEC_UP) {
+    if (i < M) {
+      if (t.c == 0) {  // routed slot: w_t * relu^2 for the slot's tokens, 0 elsewhere
+        const float* w = d.seg_w + t.e * 16;
+        __nv_bfloat16* o = d.out_up[0] + size_t(t.e) * 16 * M + i;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float wt = w[c];
+          const float a = __uint_as_float(r[c]);
+          const float v = wt != 0.f ? (a > 0.f ? a * a : 0.f) * wt : 0.f;
+          o[size_t(c) * M] = __float2bfloat16_rn(v);
+        }
+      } else {  // shared expert
+        __nv_bfloat16* o = d.out_up[1] + i;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          if (c < d.T) {
+            const float a = __uint_as_float(r[c]);
+            o[size_t(c) * M] = __float2bfloat16_rn(a > 0.f ? a * a : 0.f);
+          }
+        }
+      }
+    }
+    return;
+  }
+  // EPI_DEC_DOWN: partial of this segment, then the last of the tile's
+  // segments to arrive sums them in segment order and adds the residual.
+  if (i < M) {
+    float4* o = reinterpret_cast<float4*>(d.partial + (size_t(t.e) * M + i) * 16);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      o[c] = make_float4(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1]),
+                         __uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3]));
+  }
+  __threadfence();
+  named_barrier(1, 4 * 32);
+  const int mt = t.row0 / kBM;
+  const int nseg = *d.n_segments;
+  if (threadIdx.x == 2 * 32) last_flag = atomicAdd(d.mt_counter + mt, 1u) == unsigned(nseg - 1);
+  named_barrier(1, 4 * 32);
+  if (!last_flag) return;
+  __threadfence();
+  if (i < M) {
+    for (int c = 0; c < d.T; ++c) {
+      float acc = __bfloat162float(d.residual[size_t(c) * M + i]);
+      for (int sg = 0; sg < nseg; ++sg) acc += __ldcg(d.partial + (size_t(sg) * M + i) * 16 + c);
+      d.hidden[size_t(c) * M + i] = __float2bfloat16_rn(acc);
+    }
+  }
+  if (threadIdx.x == 2 * 32) d.mt_counter[mt] = 0u;
+  (void)lane;
 }
 
 template <int BN, int STAGES>
@@ -154,11 +232,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above overlaps the previous kernel when launched with PDL;
+  // nothing it wrote is read before this point.
+  pdl_trigger();
+  pdl_wait();
 
-  const int m0 = p.n_mtiles ? *p.n_mtiles : p.cls[0].mtiles;
-  const int W0 = m0 * p.cls[0].ntiles;
-  const int W1 = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
-  const int W = W0 + W1;
+  int W0, W;
+  if (p.dec_tiles) {
+    W0 = W = *p.dec_count;
+  } else {
+    const int m0 = p.n_mtiles ? *p.n_mtiles : p.cls[0].mtiles;
+    W0 = m0 * p.cls[0].ntiles;
+    const int W1 = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
+    W = W0 + W1;
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -183,7 +270,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&full[stage], Tr::kStageBytes);
           const int kx = kb * bk;
           const int kbx = C.b_kwrap ? (kx % C.b_kwrap) : kx;
-          tma_load_2d(sa, &p.tmA[t.c], &full[stage], kx, t.row0);
+          tma_load_2d(sa, &p.tmA[t.c], &full[stage], kx, t.arow);
           tma_load_2d(sb, &p.tmB[t.c], &full[stage], kbx, t.brow);
           ++issued;
           if (++stage == STAGES) {
@@ -282,7 +369,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int row = t.row0 + rloc;
       const bool rvalid = row < t.row_end;
 
-      if (C.epi == EPI_TOPK) {
+      if constexpr (BN == 16) {
+        decode_epilogue(p, t, tb, rloc, lane);
+      } else if (C.epi == EPI_TOPK) {
         // Sigmoid top-k of one token (row) over E <= BN logits.
         TopK tk;
         tk.init();
@@ -390,12 +479,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 template <int BN, int STAGES>
-cudaError_t launch_impl(const GemmParams& p, int grid, cudaStream_t stream) {
+cudaError_t launch_impl(const GemmParams& p, int grid, cudaStream_t stream, bool pdl) {
   using Tr = Traits<BN, STAGES>;
-  auto kern = grouped_gemm_kernel<BN, STAGES>;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kGemmThreads, Tr::kSmem, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = Tr::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, STAGES>, p);
 }
 
 template <int BN, int STAGES>
@@ -409,13 +506,16 @@ cudaError_t prepare_impl() {
 
 cudaError_t prepare_grouped_gemm() {
   cudaError_t e;
+  if ((e = prepare_impl<16, 11>()) != cudaSuccess) return e;
   if ((e = prepare_impl<128, 6>()) != cudaSuccess) return e;
   return prepare_impl<256, 4>();
 }
 
-cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStream_t stream) {
-  if (bn == 128) return launch_impl<128, 6>(p, grid, stream);
-  if (bn == 256) return launch_impl<256, 4>(p, grid, stream);
+cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStream_t stream,
+                                bool pdl) {
+  if (bn == 16) return launch_impl<16, 11>(p, grid, stream, pdl);
+  if (bn == 128) return launch_impl<128, 6>(p, grid, stream, pdl);
+  if (bn == 256) return launch_impl<256, 4>(p, grid, stream, pdl);
   return cudaErrorInvalidValue;
 }
 

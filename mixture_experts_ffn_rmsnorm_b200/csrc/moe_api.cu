@@ -114,6 +114,7 @@ struct moe_handle {
   CUtensorMap tm_up_a, tm_up_b, tm_sup_a, tm_sup_b;
   CUtensorMap tm_down_a, tm_down_b, tm_sdown_a, tm_sdown_b;
   CUtensorMap tm_fc2_a, tm_fc2_b;
+  CUtensorMap tm_dec_x, tm_dec_ub, tm_dec_vb;  // decode B operands (16-row boxes)
 };
 
 namespace {
@@ -234,6 +235,13 @@ bool build_maps(moe_handle* h) {
   ok &= make_map(&h->tm_down_b, h->w.down_w, f8, I, E * D, I * eb, 128);
   ok &= make_map(&h->tm_sdown_a, h->v, false, S, Tm, S * 2, moe::kBM);
   ok &= make_map(&h->tm_sdown_b, h->w.shared_down_w, false, S, H, S * 2, 128);
+  if (moe::decode_supported(c)) {
+    const uint64_t U = moe::decode_max_slots(c);
+    ok &= make_map(&h->tm_dec_x, h->dec.x16, false, H, moe::kDecodeN, H * 2, moe::kDecodeN);
+    ok &= make_map(&h->tm_dec_ub, h->dec.ub, false, I, (U + 1) * moe::kDecodeN, I * 2,
+                   moe::kDecodeN);
+    ok &= make_map(&h->tm_dec_vb, h->dec.vb, false, S, moe::kDecodeN, S * 2, moe::kDecodeN);
+  }
   return ok;
 }
 
@@ -380,6 +388,66 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   return MOE_OK;
 }
 
+// Decode path (T <= 8): CUDA-core routing kernel, then two tcgen05 launches
+// with the weights as the 128-row operand and the tokens as N = 16, all
+// chained with programmatic dependent launch.
+moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cudaStream_t st,
+                          moe::LaunchLog* log) {
+  const moe_config& c = h->cfg;
+  if (!moe::decode_supported(c) || T < 1 || T > MOE_DECODE_MAX_TOKENS)
+    return MOE_ERR_INVALID_CONFIG;
+  const int H = c.hidden_size, I = c.moe_inter, S = c.shared_inter;
+  moe::DecodeRouteArgs ra;
+  ra.cfg = &c;
+  ra.w = &h->w;
+  ra.ws = &h->dec;
+  ra.hidden = hidden;
+  ra.residual = residual;
+  ra.T = T;
+  MOE_TRY(moe::launch_decode_route(ra, st));
+  log->done(st);
+
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.tmA[0] = h->tm_up_b;    // routed up weights [E*I, H] as the 128-row operand
+  p.tmB[0] = h->tm_dec_x;   // tokens [16, H]
+  p.tmA[1] = h->tm_sup_b;   // shared up weights [S, H]
+  p.tmB[1] = h->tm_dec_x;
+  p.cls[0] = dense_class(H, moe::kDecodeN, 0, moe::EPI_DEC_UP, nullptr, 0, moe::kDecodeN);
+  p.cls[1] = dense_class(H, moe::kDecodeN, 0, moe::EPI_DEC_UP, nullptr, 0, moe::kDecodeN);
+  p.nclasses = 2;
+  p.dec_tiles = h->dec.tiles_up;
+  p.dec_count = h->dec.n_tiles_up;
+  p.dec.T = T;
+  p.dec.M[0] = I;
+  p.dec.M[1] = S;
+  p.dec.seg_w = h->dec.seg_w;
+  p.dec.out_up[0] = h->dec.ub;
+  p.dec.out_up[1] = h->dec.vb;
+  p.status = h->status;
+  MOE_TRY(moe::launch_grouped_gemm(p, moe::kDecodeN, h->num_sms, st, true));
+  log->done(st);
+
+  p.tmA[0] = h->tm_down_b;   // routed down weights [E*H, I]
+  p.tmB[0] = h->tm_dec_ub;   // w * relu^2(up) per segment [(U+1)*16, I]
+  p.tmA[1] = h->tm_sdown_b;  // shared down weights [H, S]
+  p.tmB[1] = h->tm_dec_vb;   // [16, S]
+  p.cls[0] = dense_class(I, moe::kDecodeN, 0, moe::EPI_DEC_DOWN, nullptr, 0, moe::kDecodeN);
+  p.cls[1] = dense_class(S, moe::kDecodeN, 0, moe::EPI_DEC_DOWN, nullptr, 0, moe::kDecodeN);
+  p.dec_tiles = h->dec.tiles_down;
+  p.dec_count = h->dec.n_tiles_down;
+  p.dec.M[0] = H;
+  p.dec.M[1] = H;
+  p.dec.partial = h->dec.partial;
+  p.dec.mt_counter = h->dec.mt_counter;
+  p.dec.n_segments = h->dec.n_segments;
+  p.dec.residual = residual;
+  p.dec.hidden = hidden;
+  MOE_TRY(moe::launch_grouped_gemm(p, moe::kDecodeN, h->num_sms, st, true));
+  log->done(st);
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -483,14 +551,8 @@ moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t
                       (path == MOE_PATH_AUTO && num_tokens <= MOE_DECODE_MAX_TOKENS &&
                        moe::decode_supported(h->cfg));
   if (decode) {
-    moe::DecodeArgs a;
-    a.cfg = &h->cfg;
-    a.w = &h->w;
-    a.ws = &h->dec;
-    a.status = h->status;
-    a.num_sms = h->num_sms;
-    st = moe::enqueue_decode(a, static_cast<bf16*>(hidden), static_cast<bf16*>(residual),
-                             num_tokens, s, &log);
+    st = enqueue_decode(h, static_cast<bf16*>(hidden), static_cast<bf16*>(residual), num_tokens,
+                        s, &log);
   } else {
     st = enqueue_prefill(h, static_cast<bf16*>(hidden), static_cast<bf16*>(residual), num_tokens,
                          s, &log);
@@ -562,7 +624,7 @@ moe_status moe_copy_routing(moe_handle* h, int32_t* idx, float* w, int32_t num_t
   if (num_tokens < 1 || num_tokens != h->last_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t n = size_t(num_tokens) * h->cfg.top_k;
-  const int32_t* si = h->last_decode ? h->dec.idx : h->idx;
+  const int32_t* si = h->last_decode ? h->dec.idx : h->idx;  // written by decode_route
   const float* sw = h->last_decode ? h->dec.w : h->wts;
   MOE_TRY(cudaMemcpyAsync(idx, si, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
   MOE_TRY(cudaMemcpyAsync(w, sw, n * sizeof(float), cudaMemcpyDeviceToDevice, s));

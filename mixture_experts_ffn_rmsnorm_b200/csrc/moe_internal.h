@@ -19,21 +19,55 @@ enum EpiKind : int {
   EPI_F32 = 2,         // out = acc (float32)
   EPI_TOPK = 3,        // sigmoid top-k routing of the row (gate logits never stored)
   EPI_BLEND = 4,       // out = bf16(acc + blend_s + blend_res)  (LatentMoE fc2)
+  EPI_DEC_UP = 5,      // decode, weights x tokens: relu^2 (x routing weight) -> token-major rows
+  EPI_DEC_DOWN = 6,    // decode, weights x tokens: fp32 partial per segment, last arriver sums
+};
+
+// Decode tiles multiply 128 weight rows (A) by the <= 16 token vectors (B,
+// N = 16) of one segment: a routed expert slot or the shared expert.
+struct DecodeTile {
+  int cls;    // class (0 routed, 1 shared)
+  int seg;    // segment: 0 = shared expert, 1 + s = routed slot s
+  int arow;   // first A row (weight row, expert offset included)
+  int brow;   // first B row (token group)
+  int m0;     // first output row of the tile inside its segment's matrix
+};
+
+struct DecodeEpilogue {
+  int T;                       // tokens (<= 8)
+  int M[2];                    // output rows per class (I or S for up, H for down)
+  const float* seg_w;          // [segments, 16] routing weight of token t (0 if not routed)
+  __nv_bfloat16* out_up[2];    // up: [segments-or-1, 16, M] token-major relu^2 rows
+  float* partial;              // down: [segments, M, 16]
+  unsigned* mt_counter;        // down: arrivals per 128-row tile (self-resetting)
+  const int* n_segments;       // down: segments of the step (device)
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* hidden;       // [T, H]
 };
 
 // Counts the kernels a call enqueues and, when profiling is enabled, records
 // caller-owned CUDA events around them: events[0] before the first launch,
 // events[i] after the i-th.
+// While the stream is being captured into a CUDA graph the events are
+// recorded as external event nodes, so they time every replay.
 struct LaunchLog {
   int count = 0;
   void* const* events = nullptr;
   int nevents = 0;
-  void begin(cudaStream_t s) const {
-    if (nevents > 0) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s);
+  unsigned flags = cudaEventRecordDefault;
+  void record(int i, cudaStream_t s) const {
+    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), s, flags);
+  }
+  void begin(cudaStream_t s) {
+    if (nevents <= 0) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+      flags = cudaEventRecordExternal;
+    record(0, s);
   }
   void done(cudaStream_t s) {
     ++count;
-    if (count < nevents) cudaEventRecord(static_cast<cudaEvent_t>(events[count]), s);
+    if (count < nevents) record(count, s);
   }
 };
 
@@ -78,11 +112,18 @@ struct GemmParams {
   const float* blend_s;
   const __nv_bfloat16* blend_res;
   int* status;
+  // Decode mode (BN = 16): tile i is dec_tiles[i] for i < *dec_count.
+  const DecodeTile* dec_tiles;
+  const int* dec_count;
+  DecodeEpilogue dec;
 };
 
-// Launch the persistent grouped GEMM (bn = 128 or 256); the operand type is
-// a per-class property (GemmClass::fp8).
-cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStream_t stream);
+// Launch the persistent grouped GEMM (bn = 16, 128 or 256); the operand type
+// is a per-class property (GemmClass::fp8).  pdl: launch with programmatic
+// stream serialization (the kernel waits on griddepcontrol before reading
+// anything the previous kernel wrote).
+cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStream_t stream,
+                                bool pdl = false);
 // Set the dynamic shared memory limit of every GEMM instantiation on the
 // current device (call once per device before launching).
 cudaError_t prepare_grouped_gemm();
