@@ -60,7 +60,7 @@ def measured_peaks():
 
 # ------------------------------------------------------- work per kernel ---
 
-def stage_model(s, T, path, U):
+def stage_model(s, T, path, U, router_split=False):
     """Algorithmic bytes / flops of every kernel the chosen path launches.
 
     U = distinct routed experts of the step (weights touched once each).
@@ -82,11 +82,18 @@ def stage_model(s, T, path, U):
              2 * R * I * D + 2 * T * S * H),
         ]
     st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2 + (T * H if s.expert_fp8 else 0), 0)]
+    # With split K (few token tiles) the router GEMM stores partial logits
+    # and a second kernel sums them and selects; its algorithmic bytes are
+    # the routing table it writes (the partials are the split's overhead).
+    sel = "" if router_split else "_topk"
     if L:
-        st.append(("router_gemm_topk+fc1", E * H * 2 + T * 2 * H * 2 + L * H * 2 + T * L * 2,
+        st.append((f"router_gemm{sel}+fc1", E * H * 2 + T * 2 * H * 2 + L * H * 2 + T * L * 2,
                    2 * T * E * H + 2 * T * H * L))
     else:
-        st.append(("router_gemm_topk", E * H * 2 + T * 2 * H * 2 + R * 8, 2 * T * E * H))
+        st.append((f"router_gemm{sel}", E * H * 2 + T * 2 * H * 2 + (0 if router_split else R * 8),
+                   2 * T * E * H))
+    if router_split:
+        st.append(("router_reduce_topk", R * 8, 0))
     st += [
         ("sort", R * 4 * 3 + (E + 1) * 4, 0),
         ("gather", 2 * R * D * wb, 0),
@@ -430,6 +437,8 @@ def main():
 
     peaks = measured_peaks()
     model = stage_model(shape, T, path, U)
+    if path == "prefill" and len(model) + 1 == nl:
+        model = stage_model(shape, T, path, U, router_split=True)
     if len(model) != nl:  # keep the JSON honest if the launch list changed
         model = [(f"kernel_{j}", 0, 0) for j in range(nl)]
     mean_stage = stage_ms.mean(axis=0)

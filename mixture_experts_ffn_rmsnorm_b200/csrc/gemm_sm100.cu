@@ -21,6 +21,7 @@
 #include "moe_internal.h"
 #include "ptx.cuh"
 #include "topk.cuh"
+#include "../../include/moe_b200.h"
 
 namespace moe {
 namespace {
@@ -50,11 +51,16 @@ struct Tile {
   int n0;       // first output column
   int brow;     // first B row
   int arow;     // first A row to load
+  int split;    // K split index (dense classes)
+  int k0, k1;   // K-block range [k0, k1); k1 < 0 = through the end
 };
 
 template <int BN>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w, int W0) {
   Tile t;
+  t.split = 0;
+  t.k0 = 0;
+  t.k1 = -1;
   if (p.dec_tiles) {
     const DecodeTile d = p.dec_tiles[w];
     t.c = d.cls;
@@ -67,9 +73,19 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w, int W0) 
     return t;
   }
   if (w < W0) {
-    const int nt = p.cls[0].ntiles;
+    const int ks = p.cls[0].ksplit > 1 ? p.cls[0].ksplit : 1;
+    const int nt = p.cls[0].ntiles * ks;
     const int mt = w / nt;
-    const int ni = w - mt * nt;
+    int ni = w - mt * nt;
+    if (ks > 1) {
+      t.split = ni % ks;
+      ni /= ks;
+      const int bk = p.cls[0].fp8 ? 128 : 64;
+      const int nk = (p.cls[0].K + bk - 1) / bk;
+      const int per = (nk + ks - 1) / ks;
+      t.k0 = t.split * per;
+      t.k1 = min(nk, t.k0 + per);
+    }
     t.c = 0;
     if (p.tile_table) {
       const int2 te = p.tile_table[mt];
@@ -119,6 +135,70 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
 __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort) {
   *abort = 1;
   if (p.status) atomicOr(p.status, kStatusWaitTimeout);
+}
+
+// Router epilogue: one thread per token row holds its E <= BN logits.
+// Without split K the thread runs the sigmoid top-k itself and the tile's
+// expert histogram (for the sort) is accumulated in shared memory and
+// written out.  With split K every split only stores its fp32 partial
+// logits, row-major [split][row][E], for the reduction kernel.
+template <int BN>
+__device__ __forceinline__ void router_epilogue(const GemmParams& p, const GemmClass& C,
+                                                const Tile& t, uint32_t tb, int row,
+                                                bool rvalid) {
+  __shared__ int s_hist[MOE_MAX_EXPERTS];
+  const int E = p.num_experts;
+  const int ep = threadIdx.x - 2 * 32;  // 0..127 inside the epilogue warps
+  if (C.ksplit > 1) {
+    float* prow = p.topk_part + (size_t(t.split) * p.topk_rows_cap + row) * E;
+    const bool vec = (E & 3) == 0;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tb + uint32_t(c * 32), r);
+      tmem_ld_wait();
+      if (rvalid) {
+        if (vec) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            if (c * 32 + j < E)
+              *reinterpret_cast<float4*>(prow + c * 32 + j) =
+                  make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                              __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < E) prow[c * 32 + j] = __uint_as_float(r[j]);
+        }
+      }
+    }
+    return;
+  }
+  TopK tk;
+  tk.init();
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tb + uint32_t(c * 32), r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = c * 32 + j;
+      if (e < E) tk.offer(e, __uint_as_float(r[j]), p.gate_bias ? p.gate_bias[e] : 0.0f, p.top_k);
+    }
+  }
+  const int mt = t.row0 / kBM;
+  for (int e = ep; e < E; e += 4 * 32) s_hist[e] = 0;
+  named_barrier(1, 4 * 32);
+  if (rvalid) {
+    tk.write(p.top_k, p.rsf, p.topk_idx + size_t(row) * p.top_k, p.topk_w + size_t(row) * p.top_k);
+#pragma unroll
+    for (int j = 0; j < kTopKMax; ++j)  // (an unfilled slot, id -1, only with NaN logits)
+      if (j < p.top_k && unsigned(tk.id[j]) < unsigned(E)) atomicAdd(&s_hist[tk.id[j]], 1);
+  }
+  named_barrier(1, 4 * 32);
+  if (p.expert_hist)
+    for (int e = ep; e < E; e += 4 * 32) p.expert_hist[size_t(mt) * E + e] = s_hist[e];
 }
 
 // Decode epilogues (BN = 16: 128 weight rows x 16 token columns).
@@ -242,7 +322,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     W0 = W = *p.dec_count;
   } else {
     const int m0 = p.n_mtiles ? *p.n_mtiles : p.cls[0].mtiles;
-    W0 = m0 * p.cls[0].ntiles;
+    W0 = m0 * p.cls[0].ntiles * (p.cls[0].ksplit > 1 ? p.cls[0].ksplit : 1);
     const int W1 = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
     W = W0 + W1;
   }
@@ -258,8 +338,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const Tile t = decode_tile<BN>(p, w, W0);
         const GemmClass& C = p.cls[t.c];
         const int bk = stage_k(C);
-        const int nk = (C.K + bk - 1) / bk;
-        for (int kb = 0; kb < nk; ++kb) {
+        const int nk = t.k1 >= 0 ? t.k1 : (C.K + bk - 1) / bk;
+        for (int kb = t.k0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) {
             record_timeout(p, abort);
             ok = false;
@@ -309,7 +389,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const Tile t = decode_tile<BN>(p, w, W0);
         const bool f8 = p.cls[t.c].fp8 != 0;
         const int bk = f8 ? 128 : 64;
-        const int nk = (p.cls[t.c].K + bk - 1) / bk;
+        const int nk = t.k1 >= 0 ? t.k1 : (p.cls[t.c].K + bk - 1) / bk;
         const int ab = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[ab], aph ^ 1u, abort)) {
@@ -318,7 +398,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(ab * BN);
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = t.k0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort)) {
             record_timeout(p, abort);
             ok = false;
@@ -331,7 +411,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < Tr::kKSteps; ++kk) {
             const uint64_t koff = uint64_t((kk * 32) >> 4);
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            const uint32_t acc = (kb != t.k0 || kk != 0) ? 1u : 0u;
             if (f8)
               umma_f8(d, ad + koff, bd + koff, idesc_f8, acc);
             else
@@ -372,24 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if constexpr (BN == 16) {
         decode_epilogue(p, t, tb, rloc, lane);
       } else if (C.epi == EPI_TOPK) {
-        // Sigmoid top-k of one token (row) over E <= BN logits.
-        TopK tk;
-        tk.init();
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tb + uint32_t(c * 32), r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int e = c * 32 + j;
-            if (e < p.num_experts)
-              tk.offer(e, __uint_as_float(r[j]), p.gate_bias ? p.gate_bias[e] : 0.0f, p.top_k);
-          }
-        }
-        if (rvalid)
-          tk.write(p.top_k, p.rsf, p.topk_idx + size_t(row) * p.top_k,
-                   p.topk_w + size_t(row) * p.top_k);
+        router_epilogue<BN>(p, C, t, tb, row, rvalid);
       } else {
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {

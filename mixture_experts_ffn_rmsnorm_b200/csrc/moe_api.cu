@@ -88,6 +88,8 @@ struct moe_handle {
   float* wts;      // [Tm*k]  (immediately after idx, as the pages' scratch layout)
   int32_t* off;    // [E+1]
   int2* tiles;     // [Rm/128 + E]
+  float* topk_part;        // [sms * 128, E] router split-K partial logits
+  int32_t* expert_hist;    // [ceil(Tm/128), E]
   int32_t* n_mtiles;
   int32_t* status;
   int32_t* perm;   // [Rm]
@@ -182,6 +184,8 @@ void carve(moe_handle* h, char* base) {
   h->wts = cv.take<float>(Rm);
   h->off = cv.take<int32_t>(E + 1);
   h->tiles = cv.take<int2>(Rm / moe::kBM + E + 1);
+  h->topk_part = cv.take<float>(size_t(h->num_sms) * moe::kBM * E);
+  h->expert_hist = cv.take<int32_t>((Tm + moe::kBM - 1) / moe::kBM * E);
   h->n_mtiles = cv.take<int32_t>(1);
   h->status = cv.take<int32_t>(1);
   h->perm = cv.take<int32_t>(Rm);
@@ -264,14 +268,14 @@ moe::GemmClass dense_class(int K, int N, int rows, int epi, void* out, int ldo, 
     if (_e != cudaSuccess) return MOE_ERR_CUDA;        \
   } while (0)
 
-// Norm + router GEMM with fused top-k (+ fc1 for LatentMoE).
+// Norm + router GEMM with fused top-k (+ fc1 for LatentMoE).  When the
+// token tiles alone would leave most SMs idle, the router's K (2H) is split
+// so that tiles x splits fill the SMs left by the other class: every split
+// stores fp32 partial logits and a second kernel sums them in split order
+// and selects (one warp per token).
 moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int T,
                          bool with_fc1, cudaStream_t st, moe::LaunchLog* log) {
   const moe_config& c = h->cfg;
-  MOE_TRY(moe::launch_rmsnorm(hidden, static_cast<const bf16*>(h->w.norm_w), residual, h->gate_a,
-                              h->fp8 && with_fc1 ? h->nq : nullptr, h->nq_scale, T,
-                              c.hidden_size, c.rms_eps, st));
-  log->done(st);
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.tmA[0] = h->tm_gate_a;
@@ -288,6 +292,26 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
                            h->gate_bn);
     p.nclasses = 2;
   }
+  const int mt = p.cls[0].mtiles;
+  int ks = 1;
+  if (c.num_experts <= 256) {
+    const int nk = (2 * c.hidden_size + 63) / 64;
+    const int other = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
+    ks = h->num_sms > other ? (h->num_sms - other) / mt : 1;
+    ks = ks < 1 ? 1 : (ks > moe::kRouterMaxSplit ? moe::kRouterMaxSplit : ks);
+    ks = ks > nk ? nk : ks;
+    const int per = (nk + ks - 1) / ks;
+    ks = (nk + per - 1) / per;  // every split non-empty
+  }
+  p.cls[0].ksplit = ks;
+  MOE_TRY(moe::launch_rmsnorm(hidden, static_cast<const bf16*>(h->w.norm_w), residual, h->gate_a,
+                              h->fp8 && with_fc1 ? h->nq : nullptr, h->nq_scale, T,
+                              c.hidden_size, c.rms_eps, ks > 1 ? h->expert_hist : nullptr,
+                              mt * c.num_experts, st));
+  log->done(st);
+  p.topk_part = h->topk_part;
+  p.topk_rows_cap = mt * moe::kBM;
+  p.expert_hist = h->expert_hist;
   p.gate_bias = h->w.gate_bias;
   p.top_k = c.top_k;
   p.num_experts = c.num_experts;
@@ -295,10 +319,16 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
   p.topk_idx = h->idx;
   p.topk_w = h->wts;
   p.status = h->status;
-  int W = p.cls[0].mtiles + (p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0);
+  int W = mt * ks + (p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0);
   const int grid = W < h->num_sms ? W : h->num_sms;
   MOE_TRY(moe::launch_grouped_gemm(p, h->gate_bn, grid, st));
   log->done(st);
+  if (ks > 1) {
+    MOE_TRY(moe::launch_router_reduce(h->topk_part, ks, mt * moe::kBM, T, c.num_experts,
+                                      h->w.gate_bias, c.top_k, c.routed_scaling_factor, h->idx,
+                                      h->wts, h->expert_hist, st));
+    log->done(st);
+  }
   return MOE_OK;
 }
 
@@ -309,8 +339,8 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
             S = c.shared_inter, L = c.latent_size, D = h->D, R = T * k;
   moe_status rs = enqueue_route(h, hidden, residual, T, true, st, log);
   if (rs != MOE_OK) return rs;
-  MOE_TRY(moe::launch_sort(h->idx, T, k, E, h->perm, h->inv, h->off, h->tiles, h->n_mtiles,
-                           h->status, st));
+  MOE_TRY(moe::launch_sort(h->idx, h->expert_hist, T, k, E, h->perm, h->inv, h->off, h->tiles,
+                           h->n_mtiles, h->status, st));
   log->done(st);
   if (L)
     MOE_TRY(moe::launch_gather(h->z, size_t(L) * 2, h->perm, k, R, D * 2, h->xs, nullptr,
@@ -610,9 +640,12 @@ moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_tokens, int32
   if (st != MOE_OK) return st;
   if (!idx || !perm || !inv || !off) return MOE_ERR_NULL_POINTER;
   if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
-  MOE_TRY(moe::launch_sort(idx, num_tokens, h->cfg.top_k, h->cfg.num_experts, perm, inv, off,
-                           h->tiles, h->n_mtiles, h->status, static_cast<cudaStream_t>(stream)));
-  h->last_launches = 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(moe::launch_tile_hist(idx, num_tokens, h->cfg.top_k, h->cfg.num_experts,
+                                h->expert_hist, h->status, s));
+  MOE_TRY(moe::launch_sort(idx, h->expert_hist, num_tokens, h->cfg.top_k, h->cfg.num_experts,
+                           perm, inv, off, h->tiles, h->n_mtiles, h->status, s));
+  h->last_launches = 2;
   return MOE_OK;
 }
 

@@ -81,6 +81,7 @@ struct GemmClass {
   int mtiles;             // m-tiles of a dense class (ignored when the launch has a tile table)
   int rows;               // valid A rows of a dense class
   int b_kwrap;            // B's k coordinate is taken modulo this (0 = no wrap)
+  int ksplit;             // dense classes: K-block ranges per output tile (0 or 1 = whole K)
   int epi;                // EpiKind
   void* out;              // output base
   int ldo;                // output row stride in elements
@@ -108,6 +109,9 @@ struct GemmParams {
   float rsf;
   int* topk_idx;
   float* topk_w;
+  float* topk_part;        // split-K partial logits [ksplit][topk_rows_cap][E]
+  int topk_rows_cap;
+  int* expert_hist;        // [token tiles][E] experts chosen by each 128-token tile
   // EPI_BLEND
   const float* blend_s;
   const __nv_bfloat16* blend_res;
@@ -130,12 +134,27 @@ cudaError_t prepare_grouped_gemm();
 
 // Routing / sort / data movement kernels (route.cu).
 // normed_q/normed_scale (nullable): per-token E4M3 copy of the normed rows.
+// hist_clear[0..n_clear) is zeroed on the way (the split-K router's
+// histogram, accumulated with atomics); may be null.
 cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* norm_w,
                            __nv_bfloat16* residual, __nv_bfloat16* gate_a, uint8_t* normed_q,
-                           float* normed_scale, int T, int H, float eps, cudaStream_t stream);
-size_t sort_smem_bytes(int E);
-cudaError_t launch_sort(const int* idx, int T, int k, int E, int* perm, int* inv, int* off,
-                        int2* tile_table, int* n_mtiles, int* status, cudaStream_t stream);
+                           float* normed_scale, int T, int H, float eps, int* hist_clear,
+                           int n_clear, cudaStream_t stream);
+// Split-K router, second half: logits = sum of the ks partials in split
+// order, sigmoid top-k per token into idx/w, and hist[t / 128][e] += 1 for
+// every chosen expert (hist zeroed beforehand).  Launched as a programmatic
+// dependent of the router GEMM.
+constexpr int kRouterMaxSplit = 16;
+cudaError_t launch_router_reduce(const float* part, int ks, int rows_cap, int T, int E,
+                                 const float* bias, int k, float rsf, int* idx, float* w,
+                                 int* hist, cudaStream_t stream);
+// Stable sort by expert from the routing table idx [T, k] and its per-128-
+// token-tile expert histogram hist [ceil(T/128), E].
+cudaError_t launch_tile_hist(const int* idx, int T, int k, int E, int* hist, int* status,
+                             cudaStream_t stream);
+cudaError_t launch_sort(const int* idx, const int* hist, int T, int k, int E, int* perm, int* inv,
+                        int* off, int2* tile_table, int* n_mtiles, int* status,
+                        cudaStream_t stream);
 // Row gather: xs[p] = X[perm[p] / k] (row_bytes per row; ldx_bytes source
 // stride); optionally scales: xs_scale[p] = scale[perm[p] / k].
 cudaError_t launch_gather(const void* X, size_t ldx_bytes, const int* perm, int k, int R,

@@ -4,8 +4,10 @@
 // expert and the residual add.
 #include <cuda_fp8.h>
 
+#include "../../include/moe_b200.h"
 #include "moe_internal.h"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace moe {
 namespace {
@@ -67,13 +69,16 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 // and lo = bf16(n - hi), so the router GEMM on [hi | lo] x [G | G] sees n to
 // about 16 significant bits (FP32-accurate logits from BF16 tensor cores).
 // With FP8 experts it also writes an E4M3 copy of n with one float scale per
-// token (scale = max|n| / 448).
+// token (scale = max|n| / 448).  hist_clear[0..n_clear) is zeroed.
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ norm_w,
     __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ gate_a,
-    uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale, int H, float eps) {
+    uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale, int H, float eps,
+    int* __restrict__ hist_clear, int n_clear) {
   __shared__ float red[kNormThreads / 32];
   const int t = blockIdx.x;
+  for (int i = t * kNormThreads + threadIdx.x; i < n_clear; i += gridDim.x * kNormThreads)
+    hist_clear[i] = 0;
   const uint4* x = reinterpret_cast<const uint4*>(hidden + size_t(t) * H);
   uint4* res = reinterpret_cast<uint4*>(residual + size_t(t) * H);
   const int nv = H / 8;
@@ -121,6 +126,46 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
   }
 }
 
+// Split-K router, second half (one warp per token).  Lane l sums the
+// partial logits of experts l, l + 32, ... over the splits in split order
+// (all loads of a group of 8 splits in flight, each warp load one coalesced
+// 128-byte row segment), then the warp runs the sigmoid top-k on the sums
+// and adds the token's choices to its 128-token tile's expert histogram.
+__global__ void __launch_bounds__(256) router_reduce_kernel(
+    const float* __restrict__ part, int ks, int rows_cap, int T, int E,
+    const float* __restrict__ bias, int k, float rsf, int* __restrict__ idx,
+    float* __restrict__ w, int* __restrict__ hist) {
+  pdl_wait();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  const size_t sstride = size_t(rows_cap) * E;
+  const float* src = part + size_t(t) * E + lane;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+#pragma unroll
+  for (int s0 = 0; s0 < kRouterMaxSplit; s0 += 8) {
+    if (s0 < ks) {
+      float v[8][8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[s][j] = (s0 + s < ks && lane + 32 * j < E)
+                        ? __ldcg(src + size_t(s0 + s) * sstride + 32 * j)
+                        : 0.f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += v[s][j];
+    }
+  }
+  const int e = warp_topk_regs(acc, bias, E, k, rsf, idx + size_t(t) * k, w + size_t(t) * k);
+  // (an out-of-range id comes only from NaN logits; the sort flags it)
+  if (lane < k && unsigned(e) < unsigned(E)) atomicAdd(hist + size_t(t / kBM) * E + e, 1);
+}
+
 // uq[p] = E4M3(u[p] / s_p), s_p = amax_p / 448; amax_p reset to 0 for the
 // next forward.  One block per row.
 __global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ u,
@@ -145,84 +190,133 @@ __global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ u,
   }
 }
 
-constexpr int kSortThreads = 1024;
+constexpr int kSortThreads = 512;
 constexpr int kSortWarps = kSortThreads / 32;
 
-// Stable sort of the R = T*k routed rows by expert in one CTA: per-warp
-// expert histograms over contiguous row segments, an exclusive prefix over
-// (expert, warp), then each warp scatters its segment 32 rows at a time,
-// ranking equal experts inside the batch with __match_any_sync so row order
-// is kept within every expert.  Also emits the m-tile table of the grouped
-// GEMM: ceil(count_e / 128) tiles per expert, in expert order.
-__global__ void __launch_bounds__(kSortThreads) sort_kernel(
-    const int* __restrict__ idx, int R, int E, int* __restrict__ perm, int* __restrict__ inv,
-    int* __restrict__ off, int2* __restrict__ tile_table, int* __restrict__ n_mtiles,
-    int* __restrict__ status) {
-  extern __shared__ int sm[];
-  int* hist = sm;                      // [kSortWarps][E]: counts, then write cursors
-  int* eoff = hist + kSortWarps * E;   // [E + 1]
-  int* toff = eoff + E + 1;            // [E + 1]
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kSortWarps * E; i += kSortThreads) hist[i] = 0;
+// Expert histogram of each 128-token tile of a routing table (the router
+// GEMM's epilogue produces the same table during a forward pass).
+__global__ void tile_hist_kernel(const int* __restrict__ idx, int T, int k, int E,
+                                 int* __restrict__ hist, int* __restrict__ status) {
+  __shared__ int h[MOE_MAX_EXPERTS];
+  const int mt = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
-  const int seg = (R + kSortWarps - 1) / kSortWarps;
-  const int f0 = min(R, warp * seg);
-  const int f1 = min(R, f0 + seg);
-  for (int f = f0 + lane; f < f1; f += 32) {
+  const int f0 = mt * kBM * k, f1 = min(T, (mt + 1) * kBM) * k;
+  for (int f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
     const int e = idx[f];
     if (unsigned(e) < unsigned(E))
-      atomicAdd(&hist[warp * E + e], 1);
+      atomicAdd(&h[e], 1);
     else
       atomicOr(status, kStatusBadIndex);
   }
   __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[size_t(mt) * E + e] = h[e];
+}
+
+// Stable sort of the R = T*k routed rows by expert, one CTA per 128-token
+// tile.  From the per-tile expert histograms every CTA derives the global
+// per-expert offsets (exclusive prefix over experts) and its own base
+// (prefix over earlier tiles); inside its tile, warps take contiguous row
+// segments with per-warp histograms and scatter 32 rows at a time, ranking
+// equal experts with __match_any_sync, so rows keep token order inside every
+// expert.  CTA 0 also writes off[E + 1] and the grouped GEMM's m-tile table
+// (ceil(count_e / 128) tiles per expert, in expert order).
+__global__ void __launch_bounds__(kSortThreads) sort_tiles_kernel(
+    const int* __restrict__ idx, const int* __restrict__ hist, int T, int k, int E,
+    int* __restrict__ perm, int* __restrict__ inv, int* __restrict__ off,
+    int2* __restrict__ tile_table, int* __restrict__ n_mtiles, int* __restrict__ status) {
+  __shared__ int base[MOE_MAX_EXPERTS];
+  __shared__ int tot[MOE_MAX_EXPERTS + 1];
+  __shared__ int toff[MOE_MAX_EXPERTS + 1];
+  __shared__ int wh[kSortWarps][MOE_MAX_EXPERTS];  // per-warp counts, then cursors
+  const int mt = blockIdx.x, ntiles = gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += kSortThreads) {
-    int s = 0;
-    for (int w = 0; w < kSortWarps; ++w) s += hist[w * E + e];
-    eoff[e] = s;  // count for now
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0, tacc = 0;
-    for (int e = 0; e < E; ++e) {
-      const int c = eoff[e];
-      eoff[e] = acc;
-      toff[e] = tacc;
-      acc += c;
-      tacc += (c + kBM - 1) / kBM;
+    int before = 0, all = 0;
+    for (int m = 0; m < ntiles; ++m) {
+      const int c = hist[size_t(m) * E + e];
+      all += c;
+      if (m < mt) before += c;
     }
-    eoff[E] = acc;
-    toff[E] = tacc;
-    *n_mtiles = tacc;
+    tot[e] = all;
+    base[e] = before;
+  }
+  for (int i = threadIdx.x; i < kSortWarps * E; i += kSortThreads) wh[i / E][i % E] = 0;
+  __syncthreads();
+  if (warp == 0) {  // exclusive scans over experts: rows and 128-row tiles
+    int acc = 0, tacc = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = e < E ? tot[e] : 0;
+      int inc = c, tinc = (c + kBM - 1) / kBM;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        const int z = __shfl_up_sync(0xffffffffu, tinc, o);
+        if (lane >= o) {
+          inc += y;
+          tinc += z;
+        }
+      }
+      if (e < E) {
+        toff[e] = tacc + tinc - (c + kBM - 1) / kBM;
+        base[e] += acc + inc - c;
+        if (mt == 0) off[e] = acc + inc - c;
+      }
+      acc += __shfl_sync(0xffffffffu, inc, 31);
+      tacc += __shfl_sync(0xffffffffu, tinc, 31);
+    }
+    if (lane == 0) {
+      toff[E] = tacc;
+      if (mt == 0) {
+        off[E] = acc;
+        *n_mtiles = tacc;
+      }
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e <= E; e += kSortThreads) off[e] = eoff[e];
+  if (mt == 0) {
+    for (int e = threadIdx.x; e < E; e += kSortThreads) {
+      const int o = base[e];  // tile 0: its base is the global offset
+      for (int i = toff[e]; i < toff[e + 1]; ++i) tile_table[i] = make_int2(e, o + (i - toff[e]) * kBM);
+    }
+  }
+  // this tile's rows, in row order
+  const int f0 = mt * kBM * k, f1 = min(T, (mt + 1) * kBM) * k;
+  const int seg = (f1 - f0 + kSortWarps - 1) / kSortWarps;
+  const int g0 = min(f1, f0 + warp * seg), g1 = min(f1, g0 + seg);
+  for (int f = g0 + lane; f < g1; f += 32) {
+    const int e = idx[f];
+    if (unsigned(e) < unsigned(E)) atomicAdd(&wh[warp][e], 1);
+    else atomicOr(status, kStatusBadIndex);
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < E; e += kSortThreads) {
-    int b = eoff[e];
+    int b = base[e];
     for (int w = 0; w < kSortWarps; ++w) {
-      const int c = hist[w * E + e];
-      hist[w * E + e] = b;
+      const int c = wh[w][e];
+      wh[w][e] = b;
       b += c;
     }
-    for (int i = toff[e]; i < toff[e + 1]; ++i)
-      tile_table[i] = make_int2(e, eoff[e] + (i - toff[e]) * kBM);
   }
   __syncthreads();
-  for (int base = f0; base < f1; base += 32) {
-    const int f = base + lane;
-    const bool valid = f < f1;
-    int e = valid ? idx[f] : -1;
+  for (int g = g0; g < g1; g += 32) {
+    const int f = g + lane;
+    int e = f < g1 ? idx[f] : -1;
     if (unsigned(e) >= unsigned(E)) e = -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     if (e >= 0) {
-      const int pos = hist[warp * E + e] + rank;
-      perm[pos] = f;
-      inv[f] = pos;
+      const int pos = wh[warp][e] + rank;
+      if (pos >= 0 && pos < T * k) {
+        perm[pos] = f;
+        inv[f] = pos;
+      } else {
+        atomicOr(status, kStatusBadIndex);  // inconsistent histogram: skip the write
+      }
     }
     __syncwarp();
-    if (e >= 0 && rank == 0) hist[warp * E + e] += __popc(peers);
+    if (e >= 0 && rank == 0) wh[warp][e] += __popc(peers);
     __syncwarp();
   }
 }
@@ -305,10 +399,29 @@ __global__ void latent_reduce_kernel(const __nv_bfloat16* __restrict__ y,
 
 cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* norm_w,
                            __nv_bfloat16* residual, __nv_bfloat16* gate_a, uint8_t* normed_q,
-                           float* normed_scale, int T, int H, float eps, cudaStream_t stream) {
+                           float* normed_scale, int T, int H, float eps, int* hist_clear,
+                           int n_clear, cudaStream_t stream) {
   rmsnorm_kernel<<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, normed_q,
-                                                 normed_scale, H, eps);
+                                                 normed_scale, H, eps, hist_clear,
+                                                 hist_clear ? n_clear : 0);
   return cudaGetLastError();
+}
+
+cudaError_t launch_router_reduce(const float* part, int ks, int rows_cap, int T, int E,
+                                 const float* bias, int k, float rsf, int* idx, float* w,
+                                 int* hist, cudaStream_t stream) {
+  if (ks < 2 || ks > kRouterMaxSplit || E > 256) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((T + 7) / 8);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, router_reduce_kernel, part, ks, rows_cap, T, E, bias, k, rsf,
+                            idx, w, hist);
 }
 
 cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* amax, uint8_t* uq,
@@ -318,18 +431,17 @@ cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* amax, uint8_t
   return cudaGetLastError();
 }
 
-size_t sort_smem_bytes(int E) { return sizeof(int) * (size_t(kSortWarps) * E + 2 * (E + 1)); }
+cudaError_t launch_tile_hist(const int* idx, int T, int k, int E, int* hist, int* status,
+                             cudaStream_t stream) {
+  tile_hist_kernel<<<(T + kBM - 1) / kBM, 256, 0, stream>>>(idx, T, k, E, hist, status);
+  return cudaGetLastError();
+}
 
-cudaError_t launch_sort(const int* idx, int T, int k, int E, int* perm, int* inv, int* off,
-                        int2* tile_table, int* n_mtiles, int* status, cudaStream_t stream) {
-  const size_t smem = sort_smem_bytes(E);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
-    if (e != cudaSuccess) return e;
-  }
-  sort_kernel<<<1, kSortThreads, smem, stream>>>(idx, T * k, E, perm, inv, off, tile_table,
-                                                 n_mtiles, status);
+cudaError_t launch_sort(const int* idx, const int* hist, int T, int k, int E, int* perm, int* inv,
+                        int* off, int2* tile_table, int* n_mtiles, int* status,
+                        cudaStream_t stream) {
+  sort_tiles_kernel<<<(T + kBM - 1) / kBM, kSortThreads, 0, stream>>>(
+      idx, hist, T, k, E, perm, inv, off, tile_table, n_mtiles, status);
   return cudaGetLastError();
 }
 

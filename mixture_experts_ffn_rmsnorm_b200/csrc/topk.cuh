@@ -66,18 +66,20 @@ struct TopK {
 };
 
 // Warp-cooperative top-k of one token's E <= 256 logits (same selection rule
-// and weight formula as TopK): lane l owns experts l, l + 32, ...; k rounds
-// of a warp arg-max on (key descending, expert index ascending).  idx[0..k)
-// and w[0..k) are written by the warp (global or shared memory).
-__device__ __forceinline__ void warp_topk(const float* logits, const float* bias, int E, int k,
-                                          float rsf, int* idx, float* w) {
+// and weight formula as TopK): lane l holds the logits of experts l, l + 32,
+// ... in lg[]; k rounds of a warp arg-max on (key descending, expert index
+// ascending).  idx[0..k) and w[0..k) are written by the warp (global or
+// shared memory).  Returns, on lanes < k, the expert chosen in round `lane`
+// (-1 elsewhere).
+__device__ __forceinline__ int warp_topk_regs(const float (&lg)[8], const float* bias, int E,
+                                              int k, float rsf, int* idx, float* w) {
   const int lane = threadIdx.x & 31;
   float key[8], sc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = lane + 32 * j;
     if (e < E) {
-      const float s = 1.0f / (1.0f + expf(-__ldcg(logits + e)));
+      const float s = 1.0f / (1.0f + expf(-lg[j]));
       sc[j] = s;
       key[j] = s + (bias ? bias[e] : 0.0f);
     } else {
@@ -86,6 +88,7 @@ __device__ __forceinline__ void warp_topk(const float* logits, const float* bias
     }
   }
   float sum = 0.f, mine = 0.f;
+  int mine_e = -1;
   for (int r = 0; r < k; ++r) {
     float bk = -INFINITY;
     int be = 0x7fffffff;
@@ -119,10 +122,22 @@ __device__ __forceinline__ void warp_topk(const float* logits, const float* bias
     sum += s;
     if (lane == r) {
       mine = s;
+      mine_e = be;
       idx[r] = be;
     }
   }
   if (lane < k) w[lane] = mine * (rsf / sum);
+  return mine_e;
+}
+
+// Same, reading the logits from global memory (logits[0..E)).
+__device__ __forceinline__ void warp_topk(const float* logits, const float* bias, int E, int k,
+                                          float rsf, int* idx, float* w) {
+  const int lane = threadIdx.x & 31;
+  float lg[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) lg[j] = lane + 32 * j < E ? __ldcg(logits + lane + 32 * j) : 0.f;
+  warp_topk_regs(lg, bias, E, k, rsf, idx, w);
 }
 
 }  // namespace moe
