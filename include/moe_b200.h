@@ -177,6 +177,45 @@ MOE_API moe_status moe_route(moe_handle* h, const void* hidden, int32_t num_toke
 MOE_API moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_tokens, int32_t* perm,
                     int32_t* inv, int32_t* off, void* stream);
 
+/* Largest num_tokens moe_sort_static accepts. */
+#define MOE_SORT_STATIC_MAX_TOKENS 8192
+
+/* The same sort-by-expert as moe_sort (same outputs, bit for bit), without a
+ * handle and without allocating device memory.  The pages have no
+ * counterpart: the layer they describe always sorts inside its forward
+ * pass, from its own scratch.
+ *
+ * For callers that cannot allocate at the call: a runtime whose device
+ * memory budget is fixed up front, a thread that must not stall the device
+ * (cudaFree synchronises it), or code holding routing from elsewhere and no
+ * moe_handle.  The scratch (about 75 KB: per-tile expert histograms, the
+ * m-tile table, the status word) is a fixed array in the library's device
+ * memory, one per device.
+ *
+ *   idx [num_tokens, top_k] int32 expert ids in [0, num_experts) (device).
+ *   perm [R], inv [R], off [num_experts + 1] int32 (device, caller-owned,
+ *   R = num_tokens * top_k): as moe_sort.
+ *   status: optional device int32; set to 0, then bit 2 is OR-ed in if an
+ *   id lies outside [0, num_experts) (that row is skipped).  NULL uses a
+ *   word in the scratch.
+ *   stream: cudaStream_t (NULL = legacy default stream).
+ *
+ * Errors (nothing is launched): MOE_ERR_NULL_POINTER for a NULL idx, perm,
+ * inv or off; MOE_ERR_INVALID_CONFIG for top_k outside [1, MOE_MAX_TOP_K],
+ * num_experts outside [1, MOE_MAX_EXPERTS] or top_k > num_experts;
+ * MOE_ERR_TOKENS_OUT_OF_RANGE for num_tokens outside
+ * [1, MOE_SORT_STATIC_MAX_TOKENS]; MOE_ERR_DEVICE if the current device is
+ * not sm_100; MOE_ERR_CUDA if resolving the scratch or a launch fails.
+ *
+ * The first call on a device does set-up (it looks up the scratch array's
+ * device address, which may load the module on that device); make it before
+ * any stream capture.  The scratch is shared by all calls on a device, so
+ * calls that overlap in time there (other streams or host threads) race;
+ * the caller serialises them. */
+MOE_API moe_status moe_sort_static(const int32_t* idx, int32_t num_tokens, int32_t top_k,
+                                   int32_t num_experts, int32_t* perm, int32_t* inv, int32_t* off,
+                                   int32_t* status, void* stream);
+
 /* Copy the routing used by the last moe_forward* call on this handle (either
  * path) into idx [T, k] int32 and w [T, k] float32 (device pointers, same
  * meaning as moe_route's outputs); num_tokens must equal that call's. */

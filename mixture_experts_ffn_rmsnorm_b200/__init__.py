@@ -11,8 +11,8 @@ import ctypes
 import os
 from typing import Optional
 
-__all__ = ["load_library", "MoEConfig", "MoELayer", "MoEError", "STATUS", "PATH_AUTO",
-           "PATH_DECODE", "PATH_PREFILL", "EXPORTED_SYMBOLS", "LIB_PATH"]
+__all__ = ["load_library", "sort_static", "MoEConfig", "MoELayer", "MoEError", "STATUS",
+           "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL", "EXPORTED_SYMBOLS", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
 
@@ -27,7 +27,7 @@ WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
 EXPORTED_SYMBOLS = ("moe_create", "moe_forward", "moe_forward_path", "moe_forward_host",
                     "moe_destroy", "moe_status_string", "moe_route", "moe_sort",
                     "moe_get_device_status", "moe_last_launch_count", "moe_copy_routing",
-                    "moe_set_stage_events")
+                    "moe_set_stage_events", "moe_sort_static")
 
 
 class MoEError(RuntimeError):
@@ -81,6 +81,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_last_launch_count": ([V], I32),
         "moe_copy_routing": ([V, V, V, I32, V], ctypes.c_int),
         "moe_set_stage_events": ([V, V, I32], ctypes.c_int),
+        "moe_sort_static": ([V, I32, I32, I32, V, V, V, V, V], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -98,6 +99,18 @@ def _stream_ptr(stream) -> Optional[int]:
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
     return int(s.cuda_stream) or None
+
+
+def sort_static(idx, top_k, num_experts, perm, inv, off, status=None, stream=None):
+    """moe_sort_static: sort-by-expert of idx [T, top_k] (CUDA int32) into
+    perm, inv, off without a handle and without device allocation (scratch
+    in a fixed array of the library, at most MOE_SORT_STATIC_MAX_TOKENS
+    tokens; overlapping calls on one device race on it)."""
+    lib = load_library()
+    st = lib.moe_sort_static(_ptr(idx), idx.shape[0], top_k, num_experts, _ptr(perm), _ptr(inv),
+                             _ptr(off), _ptr(status), _stream_ptr(stream))
+    if st != 0:
+        raise MoEError(st, "moe_sort_static")
 
 
 class MoELayer:

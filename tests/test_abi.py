@@ -97,3 +97,17 @@ def test_invalid_handle_rejected():
     bogus = ctypes.create_string_buffer(64)
     assert lib.moe_forward(ctypes.addressof(bogus), None, None, 1, None) == 8
     assert lib.moe_last_launch_count(None) == -1
+
+
+def test_static_sort_validates_on_host():
+    # every rejection happens before the device is touched
+    lib = moe.load_library()
+    p = 256  # any non-NULL value: nothing is dereferenced on these paths
+    assert lib.moe_sort_static(None, 10, 2, 8, p, p, p, None, None) == 2
+    assert lib.moe_sort_static(p, 10, 2, 8, p, None, p, None, None) == 2
+    assert lib.moe_sort_static(p, 8193, 2, 8, p, p, p, None, None) == 4
+    assert lib.moe_sort_static(p, 0, 2, 8, p, p, p, None, None) == 4
+    assert lib.moe_sort_static(p, 10, 0, 8, p, p, p, None, None) == 1
+    assert lib.moe_sort_static(p, 10, 17, 64, p, p, p, None, None) == 1
+    assert lib.moe_sort_static(p, 10, 4, 257, p, p, p, None, None) == 1
+    assert lib.moe_sort_static(p, 10, 9, 8, p, p, p, None, None) == 1
