@@ -6,8 +6,8 @@
 // logit = rsqrt(mean x^2 + eps) * (G_e . (x * w)) in fp32, which is the
 // logit of the un-rounded normed vector without waiting on the norm.  The last block to
 // finish runs a warp-parallel sigmoid top-k per token, groups the routed
-// (token, slot) pairs by distinct expert into segments, and writes the tile
-// lists of the two tensor-core launches that follow.  Block 0 writes the
+// (token, slot) pairs by distinct expert into segments, and writes the
+// segment table and the up launch's tile list.  Block 0 writes the
 // residual and the bf16 normed rows (the B operand of the up launch).
 #include "decode.h"
 #include "ptx.cuh"
@@ -215,9 +215,9 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
     p.ws.seg_w[(s_seg_of[s_idx[f]] + 1) * kDecodeN + f / p.k] = s_w[f];
   const int nseg = s_nseg, nslot = nseg - 1;
   for (int s = threadIdx.x; s < nslot; s += kThreads) p.ws.seg_expert[s + 1] = s_exp[s];
-  // tile lists: shared-expert tiles first (the longest down tiles), then the
-  // routed slots, each cut into 128-row tiles
-  const int nI = (p.I + kBM - 1) / kBM, nS = (p.S + kBM - 1) / kBM, nH = (H + kBM - 1) / kBM;
+  // up tile list: shared-expert tiles first, then the routed slots, each cut
+  // into 128-row tiles (the down launch needs only the segment table)
+  const int nI = (p.I + kBM - 1) / kBM, nS = (p.S + kBM - 1) / kBM;
   for (int i = threadIdx.x; i < nS + nslot * nI; i += kThreads) {
     DecodeTile d;
     if (i < nS) {
@@ -228,18 +228,8 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
     }
     p.ws.tiles_up[i] = d;
   }
-  for (int i = threadIdx.x; i < nseg * nH; i += kThreads) {
-    const int s = i / nH, mt = i - s * nH;
-    DecodeTile d;
-    if (s == 0)
-      d = DecodeTile{1, 0, mt * kBM, 0, mt * kBM};
-    else
-      d = DecodeTile{0, s, s_exp[s - 1] * H + mt * kBM, s * kDecodeN, mt * kBM};
-    p.ws.tiles_down[i] = d;
-  }
   if (threadIdx.x == 0) {
     *p.ws.n_tiles_up = nS + nslot * nI;
-    *p.ws.n_tiles_down = nseg * nH;
     *p.ws.n_segments = nseg;
     *p.ws.counter = 0u;
   }

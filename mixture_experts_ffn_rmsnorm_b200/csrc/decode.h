@@ -6,9 +6,12 @@
 //       launches.
 //   grouped GEMM, up (tcgen05, weights x tokens, N = 16): relu^2 of every
 //       distinct routed expert's up rows and of the shared expert's.
-//   grouped GEMM, down (split by segment): every segment's down rows; the last
-//       segment of a 128-row tile to finish sums all segments in a fixed order
-//       with the residual into hidden.
+//   grouped GEMM, down: a 128-row block of the output accumulates the
+//       shared expert's and every routed slot's k-blocks in one pass
+//       (concatenated K); the last piece of the block to finish adds the
+//       pieces in k order and the residual into hidden.
+// Both GEMM launches cut their k-blocks into equal contiguous ranges, one
+// per CTA (stream-K), so every SM streams the same number of weight bytes.
 #pragma once
 
 #include <stddef.h>
@@ -33,12 +36,12 @@ struct DecodeWorkspace {
   unsigned* counter;       // [1] router blocks finished (self-resetting)
   DecodeTile* tiles_up;    // [Umax * ceil(I/128) + ceil(S/128)]
   int* n_tiles_up;         // [1]
-  DecodeTile* tiles_down;  // [(Umax + 1) * ceil(H/128)]
-  int* n_tiles_down;       // [1]
   __nv_bfloat16* ub;       // [(Umax + 1) * 16, I] w_t * relu^2(up) per segment, token-major
   __nv_bfloat16* vb;       // [16, S] shared relu^2(up), token-major
-  float* partial;          // [(Umax + 1), H, 16] down output per segment
-  unsigned* mt_counter;    // [ceil(H/128)] segments finished per row tile (self-resetting)
+  float* up_part;          // [up tiles + CTAs, 128, 16] up piece partials
+  unsigned* up_counter;    // [up tiles] pieces finished per tile (self-resetting)
+  float* partial;          // [ceil(H/128) + CTAs, 128, 16] down piece partials
+  unsigned* mt_counter;    // [ceil(H/128)] pieces finished per row tile (self-resetting)
 };
 
 inline int decode_max_slots(const moe_config& c) {
@@ -48,11 +51,14 @@ inline int decode_max_slots(const moe_config& c) {
 
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
+// ctas: grid of the decode GEMM launches (one CTA per SM).
 template <class Take>
-void carve_decode(DecodeWorkspace* d, const moe_config& c, Take take) {
+void carve_decode(DecodeWorkspace* d, const moe_config& c, int ctas, Take take) {
   const size_t k = c.top_k, E = c.num_experts, H = c.hidden_size, I = c.moe_inter,
                S = c.shared_inter;
   const size_t U = decode_max_slots(c);
+  const size_t up_tiles = U * cdiv(int(I), kBM) + cdiv(int(S), kBM);
+  const size_t down_tiles = cdiv(int(H), kBM);
   d->x16 = reinterpret_cast<__nv_bfloat16*>(take(kDecodeN * H * 2));
   d->logits = reinterpret_cast<float*>(take(kDecodeMaxT * E * 4));
   d->idx = reinterpret_cast<int*>(take(kDecodeMaxT * k * 4));
@@ -61,15 +67,13 @@ void carve_decode(DecodeWorkspace* d, const moe_config& c, Take take) {
   d->seg_w = reinterpret_cast<float*>(take((U + 1) * kDecodeN * 4));
   d->n_segments = reinterpret_cast<int*>(take(4));
   d->counter = reinterpret_cast<unsigned*>(take(4));
-  d->tiles_up = reinterpret_cast<DecodeTile*>(
-      take((U * cdiv(int(I), kBM) + cdiv(int(S), kBM)) * sizeof(DecodeTile)));
+  d->tiles_up = reinterpret_cast<DecodeTile*>(take(up_tiles * sizeof(DecodeTile)));
   d->n_tiles_up = reinterpret_cast<int*>(take(4));
-  d->tiles_down =
-      reinterpret_cast<DecodeTile*>(take((U + 1) * cdiv(int(H), kBM) * sizeof(DecodeTile)));
-  d->n_tiles_down = reinterpret_cast<int*>(take(4));
   d->ub = reinterpret_cast<__nv_bfloat16*>(take((U + 1) * kDecodeN * I * 2));
   d->vb = reinterpret_cast<__nv_bfloat16*>(take(kDecodeN * S * 2));
-  d->partial = reinterpret_cast<float*>(take((U + 1) * H * kDecodeN * 4));
+  d->up_part = reinterpret_cast<float*>(take((up_tiles + ctas) * kBM * kDecodeN * 4));
+  d->up_counter = reinterpret_cast<unsigned*>(take(up_tiles * 4));
+  d->partial = reinterpret_cast<float*>(take((down_tiles + ctas) * kBM * kDecodeN * 4));
   d->mt_counter = reinterpret_cast<unsigned*>(take(cdiv(int(H), kBM) * 4));
 }
 

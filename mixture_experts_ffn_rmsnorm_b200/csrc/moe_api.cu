@@ -207,7 +207,7 @@ void carve(moe_handle* h, char* base) {
     h->uq = cv.take<uint8_t>(Rm * I);
     h->u_scale = cv.take<float>(Rm);
   }
-  moe::carve_decode(&h->dec, c, [&](size_t bytes) { return cv.take<char>(bytes); });
+  moe::carve_decode(&h->dec, c, h->num_sms, [&](size_t bytes) { return cv.take<char>(bytes); });
   h->ws_bytes = cv.off;
 }
 
@@ -451,9 +451,12 @@ moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cu
   p.dec.T = T;
   p.dec.M[0] = I;
   p.dec.M[1] = S;
+  p.dec.n_first = (S + moe::kBM - 1) / moe::kBM;  // shared tiles lead the list
   p.dec.seg_w = h->dec.seg_w;
   p.dec.out_up[0] = h->dec.ub;
   p.dec.out_up[1] = h->dec.vb;
+  p.dec.up_part = h->dec.up_part;
+  p.dec.up_counter = h->dec.up_counter;
   p.status = h->status;
   MOE_TRY(moe::launch_grouped_gemm(p, moe::kDecodeN, h->num_sms, st, true));
   log->done(st);
@@ -464,10 +467,13 @@ moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cu
   p.tmB[1] = h->tm_dec_vb;   // [16, S]
   p.cls[0] = dense_class(I, moe::kDecodeN, 0, moe::EPI_DEC_DOWN, nullptr, 0, moe::kDecodeN);
   p.cls[1] = dense_class(S, moe::kDecodeN, 0, moe::EPI_DEC_DOWN, nullptr, 0, moe::kDecodeN);
-  p.dec_tiles = h->dec.tiles_down;
-  p.dec_count = h->dec.n_tiles_down;
+  p.dec_tiles = nullptr;
+  p.dec_count = h->dec.n_segments;  // output tiles over the concatenated segments
+  p.dec_concat = 1;
+  p.l2_prefetch[0] = p.l2_prefetch[1] = nullptr;
   p.dec.M[0] = H;
   p.dec.M[1] = H;
+  p.dec.seg_expert = h->dec.seg_expert;
   p.dec.partial = h->dec.partial;
   p.dec.mt_counter = h->dec.mt_counter;
   p.dec.n_segments = h->dec.n_segments;
