@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
   __shared__ int s_seg_of[MOE_MAX_EXPERTS];
   __shared__ int s_exp[kMaxSeg];
   __shared__ int s_nseg;
-  pdl_trigger();
+  __shared__ float s_bias[MOE_MAX_EXPERTS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = p.H, T = p.T, nv = H / 8;
 
@@ -82,7 +82,14 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
                 ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e_row) * H + i))
                 : make_uint4(0, 0, 0, 0);
   }
+  // this thread's selection biases (stored to shared memory once the
+  // tokens are in, so the load does not hold up the wait below)
+  const float bias_r =  // (E <= 256 = kThreads)
+      p.gate_bias && int(threadIdx.x) < p.E ? __ldg(p.gate_bias + threadIdx.x) : 0.0f;
   pdl_wait();
+  // The next launch may start (its prologue overlaps the rest of this
+  // kernel) once this kernel's input is complete.
+  pdl_trigger();
 
   // 2. x * w_norm into shared memory (fp32) and the sum of squares per token;
   //    logit_e = r_t * (G_e . (x_t * w)), so the dot products need not wait
@@ -119,6 +126,7 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
     for (int w = 0; w < kWarps; ++w) v += red[w][threadIdx.x];
     rs[threadIdx.x] = rsqrtf(v / float(H) + p.eps);
   }
+  if (int(threadIdx.x) < p.E) s_bias[threadIdx.x] = bias_r;
   __syncthreads();
 
   // 3. router logits (fp32) of this warp's expert row
@@ -173,7 +181,7 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
   if (!am_last) return;
   __threadfence();
   for (int t = warp; t < T; t += kWarps)
-    warp_topk(p.ws.logits + t * p.E, p.gate_bias, p.E, p.k, p.rsf, s_idx + t * p.k,
+    warp_topk(p.ws.logits + t * p.E, p.gate_bias ? s_bias : nullptr, p.E, p.k, p.rsf, s_idx + t * p.k,
               s_w + t * p.k);
   __syncthreads();
   // segments: 0 = shared expert, 1.. = distinct routed experts in first-use

@@ -96,6 +96,10 @@ __device__ __forceinline__ DecSched dec_sched(const GemmParams& p, int count) {
   }
   s.total = s.n1 * s.kb1 + (s.ntiles - s.n1) * s.kb0;
   s.P = max((s.total + int(gridDim.x) - 1) / int(gridDim.x), kDecMinPiece);
+  // With no more tiles than CTAs and tiles of one length, every CTA takes
+  // at most one whole tile: no cut tiles, no partial sums.
+  if (!p.dec_concat && s.ntiles <= int(gridDim.x) && (s.n1 == 0 || s.kb0 == s.kb1))
+    s.P = max(s.P, s.n1 > 0 ? s.kb1 : s.kb0);
   return s;
 }
 

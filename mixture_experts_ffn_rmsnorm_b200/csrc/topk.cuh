@@ -1,6 +1,7 @@
 // Sigmoid top-k selection of one token, shared by the prefill router GEMM
-// epilogue and the decode routing kernel so both paths take identical
-// decisions in float32.
+// epilogue (TopK), the split-K router reduction and the decode routing
+// kernel (warp_topk_regs / warp_topk) so all paths take identical decisions
+// in float32.
 //
 // NemotronMoeLayer (nemotron_moe.rs module documentation): sigmoid top-k
 // routing.  Selection key = sigmoid(logit) + bias (bias for selection only);
