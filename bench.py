@@ -127,16 +127,17 @@ def roofline_of(name, nbytes, flops, ms, peaks, expert_fp8):
             "frac": round(ach / peaks["hbm_gbs"], 4)}
 
 
-def kernel_traffic(name):
-    """dram bytes per launch from the committed ncu summary, or None when the
-    kernel's source has changed since the capture."""
+def kernel_traffic(name, workload):
+    """dram bytes per launch of kernel stage `name` on `workload` ("prefill
+    T=1024") from the committed ncu summary, or None when there is no capture
+    of that pair or the kernel's source has changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
-    rec = d.get("kernels", {}).get(name)
+    rec = d.get("kernels", {}).get(f"{name}@{workload}")
     if not rec:
         return None
     src = os.path.join(ROOT, rec["source"])
@@ -454,7 +455,7 @@ def main():
     roof["algorithmic"] = nb[1] if dom["bound"] == "hbm" else nb[2]
     roof["peak_source"] = peaks["source"] + (" (burst copy)" if dom["bound"] == "hbm"
                                              else " bf16 burst")
-    roof["traffic"] = kernel_traffic(dom["kernel"])
+    roof["traffic"] = kernel_traffic(dom["kernel"], f"{shape.name} T={T}")
 
     if rank == 0:
         line = {
