@@ -148,6 +148,26 @@ def kernel_traffic(name, workload):
     return rec["dram_bytes_per_launch"] if h == rec.get("source_sha256_16") else None
 
 
+# ------------------------------------------------------------ multi-rank ---
+
+def max_over_ranks(ms, world, device):
+    """The job's time for a quantity every rank measured on its own device:
+    the slowest rank's (all-reduce MAX; with the barriers around the timed
+    region this is the only collective, the replicas share no data)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, T, steps, ms):
+    """Whole-job throughput: every rank processes its own T tokens per step."""
+    return world * T * steps / (ms * 1e-3)
+
+
 # --------------------------------------------------------------- clocks ---
 
 class ClockSampler:
@@ -394,12 +414,8 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
     step_ms = np.array([a.elapsed_time(b) for a, b in zip(e_start, e_end)])
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * T * args.steps / (total_ms * 1e-3)
+    total_ms = max_over_ranks(float(step_ms.sum()), world, "cuda")
+    value = job_tokens_per_s(world, T, args.steps, total_ms)
 
     # per-kernel device times: events recorded between the launches
     n_prof = min(args.steps, 50)
@@ -429,12 +445,8 @@ def main():
         layer.forward_host(h_host)
         e1[i].record(stream)
         stream.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = world * T * args.steps / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)), world, "cuda")
+    e2e = job_tokens_per_s(world, T, args.steps, e2e_ms)
 
     peaks = measured_peaks()
     model = stage_model(shape, T, path, U)
