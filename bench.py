@@ -130,7 +130,8 @@ def roofline_of(name, nbytes, flops, ms, peaks, expert_fp8):
 def kernel_traffic(name, workload):
     """dram bytes per launch of kernel stage `name` on `workload` ("prefill
     T=1024") from the committed ncu summary, or None when there is no capture
-    of that pair or the kernel's source has changed since."""
+    of that pair or the kernel source or launch configuration has changed
+    since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -140,12 +141,21 @@ def kernel_traffic(name, workload):
     rec = d.get("kernels", {}).get(f"{name}@{workload}")
     if not rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
+    return rec["dram_bytes_per_launch"] if sources_hash(rec["sources"]) == rec.get(
+        "sources_sha256_16") else None
+
+
+def sources_hash(paths):
+    """sha256 prefix over the kernel source and the launch configuration that
+    determine a kernel's traffic (files relative to the repository root)."""
+    h = hashlib.sha256()
     try:
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        for rel in paths:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
     except OSError:
         return None
-    return rec["dram_bytes_per_launch"] if h == rec.get("source_sha256_16") else None
+    return h.hexdigest()[:16]
 
 
 # ------------------------------------------------------------ multi-rank ---

@@ -66,6 +66,15 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 
+// Output columns per tile of the prefill up and down launches.  A CTA
+// streams 16 KB of A and BN x 128 B of B per 128-byte k-block; BN = 256
+// carries twice the tensor work of BN = 128 for 1.5x the bytes, which is
+// what the launches' in-flight depth (4 stages, 192 KB) can sustain.  Narrow
+// layers (N < 512 in a launch) keep BN = 128, which wastes fewer columns.
+inline int prefill_bn(int n_routed, int n_shared) {
+  return (n_routed >= 512 && n_shared >= 512) ? 256 : 128;
+}
+
 struct moe_handle {
   uint32_t magic;
   moe_config cfg;
@@ -115,6 +124,10 @@ struct moe_handle {
   CUtensorMap tm_gate_a, tm_gate_b, tm_fc1_a, tm_fc1_b;
   CUtensorMap tm_up_a, tm_up_b, tm_sup_a, tm_sup_b;
   CUtensorMap tm_down_a, tm_down_b, tm_sdown_a, tm_sdown_b;
+  // the same weights with up_bn / down_bn-row boxes (B operand of the
+  // prefill launches; the decode launches read them as the 128-row A operand)
+  CUtensorMap tm_up_w, tm_sup_w, tm_down_w, tm_sdown_w;
+  int up_bn, down_bn;
   CUtensorMap tm_fc2_a, tm_fc2_b;
   CUtensorMap tm_dec_x, tm_dec_ub, tm_dec_vb;  // decode B operands (16-row boxes)
 };
@@ -239,6 +252,12 @@ bool build_maps(moe_handle* h) {
   ok &= make_map(&h->tm_down_b, h->w.down_w, f8, I, E * D, I * eb, 128);
   ok &= make_map(&h->tm_sdown_a, h->v, false, S, Tm, S * 2, moe::kBM);
   ok &= make_map(&h->tm_sdown_b, h->w.shared_down_w, false, S, H, S * 2, 128);
+  h->up_bn = prefill_bn(I, S);
+  h->down_bn = prefill_bn(D, H);
+  ok &= make_map(&h->tm_up_w, h->w.up_w, f8, D, E * I, D * eb, h->up_bn);
+  ok &= make_map(&h->tm_sup_w, h->w.shared_up_w, false, H, S, H * 2, h->up_bn);
+  ok &= make_map(&h->tm_down_w, h->w.down_w, f8, I, E * D, I * eb, h->down_bn);
+  ok &= make_map(&h->tm_sdown_w, h->w.shared_down_w, false, S, H, S * 2, h->down_bn);
   if (moe::decode_supported(c)) {
     const uint64_t U = moe::decode_max_slots(c);
     ok &= make_map(&h->tm_dec_x, h->dec.x16, false, H, moe::kDecodeN, H * 2, moe::kDecodeN);
@@ -357,8 +376,8 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.tmA[0] = h->tm_up_a;
-  p.tmB[0] = h->tm_up_b;
-  p.cls[0] = dense_class(D, I, 0, moe::EPI_RELU2_BF16, h->u, I, 128);
+  p.tmB[0] = h->tm_up_w;
+  p.cls[0] = dense_class(D, I, 0, moe::EPI_RELU2_BF16, h->u, I, h->up_bn);
   if (h->fp8) {  // W8A8: acc * token scale * weight-row scale, row max for requantisation
     p.cls[0].fp8 = 1;
     p.cls[0].row_scale = h->xs_scale;
@@ -366,14 +385,14 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
     p.cls[0].row_amax = h->u_amax;
   }
   p.tmA[1] = h->tm_sup_a;
-  p.tmB[1] = h->tm_sup_b;
-  p.cls[1] = dense_class(H, S, T, moe::EPI_RELU2_BF16, h->v, S, 128);
+  p.tmB[1] = h->tm_sup_w;
+  p.cls[1] = dense_class(H, S, T, moe::EPI_RELU2_BF16, h->v, S, h->up_bn);
   p.nclasses = 2;
   p.tile_table = h->tiles;
   p.n_mtiles = h->n_mtiles;
   p.group_off = h->off;
   p.status = h->status;
-  MOE_TRY(moe::launch_grouped_gemm(p, 128, h->num_sms, st));
+  MOE_TRY(moe::launch_grouped_gemm(p, h->up_bn, h->num_sms, st));
   log->done(st);
 
   if (h->fp8) {
@@ -383,17 +402,17 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
 
   // grouped down: routed -> y (bf16, sorted rows), shared -> s (f32)
   p.tmA[0] = h->tm_down_a;
-  p.tmB[0] = h->tm_down_b;
-  p.cls[0] = dense_class(I, D, 0, moe::EPI_BF16, h->y, D, 128);
+  p.tmB[0] = h->tm_down_w;
+  p.cls[0] = dense_class(I, D, 0, moe::EPI_BF16, h->y, D, h->down_bn);
   if (h->fp8) {
     p.cls[0].fp8 = 1;
     p.cls[0].row_scale = h->u_scale;
     p.cls[0].col_scale = h->w.down_scale;
   }
   p.tmA[1] = h->tm_sdown_a;
-  p.tmB[1] = h->tm_sdown_b;
-  p.cls[1] = dense_class(S, H, T, moe::EPI_F32, h->s, H, 128);
-  MOE_TRY(moe::launch_grouped_gemm(p, 128, h->num_sms, st));
+  p.tmB[1] = h->tm_sdown_w;
+  p.cls[1] = dense_class(S, H, T, moe::EPI_F32, h->s, H, h->down_bn);
+  MOE_TRY(moe::launch_grouped_gemm(p, h->down_bn, h->num_sms, st));
   log->done(st);
 
   if (!L) {
