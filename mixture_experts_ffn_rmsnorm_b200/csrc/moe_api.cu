@@ -289,9 +289,10 @@ moe::GemmClass dense_class(int K, int N, int rows, int epi, void* out, int ldo, 
 
 // Norm + router GEMM with fused top-k (+ fc1 for LatentMoE).  When the
 // token tiles alone would leave most SMs idle, the router's K (2H) is split
-// so that tiles x splits fill the SMs left by the other class: every split
-// stores fp32 partial logits and a second kernel sums them in split order
-// and selects (one warp per token).
+// so that tiles x splits fill the SMs left by the other class (or, when fc1
+// fills them, into pieces shorter than fc1's tiles): every split stores
+// fp32 partial logits and a second kernel sums them in split order and
+// selects (one warp per token).
 moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int T,
                          bool with_fc1, cudaStream_t st, moe::LaunchLog* log) {
   const moe_config& c = h->cfg;
@@ -317,6 +318,14 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
     const int nk = (2 * c.hidden_size + 63) / 64;
     const int other = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
     ks = h->num_sms > other ? (h->num_sms - other) / mt : 1;
+    if (other >= h->num_sms) {
+      // The other class alone fills the SMs (LatentMoE fc1): cut the router
+      // tiles (K = 2H) into pieces of half the other class's K, so that no
+      // router tile is the launch's long pole.
+      const int nko = (p.cls[1].K + 63) / 64;
+      ks = 2 * ((nk + nko - 1) / nko);
+    }
+    if (ks > h->num_sms / mt) ks = h->num_sms / mt;  // capacity of the partial logits
     ks = ks < 1 ? 1 : (ks > moe::kRouterMaxSplit ? moe::kRouterMaxSplit : ks);
     ks = ks > nk ? nk : ks;
     const int per = (nk + ks - 1) / ks;

@@ -126,6 +126,87 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
   }
 }
 
+// The same RMSNorm with the token's chunks of x and of the norm weight held
+// in registers (H <= kNormThreads * 8 * MAXC): x is read from memory once and
+// the weight load overlaps it, ahead of the block reduction.  Identical
+// arithmetic and summation order, hence identical results.
+template <int MAXC>
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(
+    const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ norm_w,
+    __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ gate_a,
+    uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale, int H, float eps,
+    int* __restrict__ hist_clear, int n_clear) {
+  __shared__ float red[kNormThreads / 32];
+  const int t = blockIdx.x;
+  for (int i = t * kNormThreads + threadIdx.x; i < n_clear; i += gridDim.x * kNormThreads)
+    hist_clear[i] = 0;
+  const uint4* x = reinterpret_cast<const uint4*>(hidden + size_t(t) * H);
+  const uint4* w = reinterpret_cast<const uint4*>(norm_w);
+  uint4* res = reinterpret_cast<uint4*>(residual + size_t(t) * H);
+  const int nv = H / 8;
+  uint4 xv[MAXC], wv[MAXC];
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int i = threadIdx.x + c * kNormThreads;
+    if (i < nv) {
+      xv[c] = x[i];
+      wv[c] = w[i];
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int i = threadIdx.x + c * kNormThreads;
+    if (i < nv) {
+      res[i] = xv[c];
+      float f[8];
+      unpack8(xv[c], f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss += f[j] * f[j];
+    }
+  }
+  const float r = rsqrtf(block_reduce(ss, red, false) / float(H) + eps);
+  uint4* hi = reinterpret_cast<uint4*>(gate_a + size_t(t) * 2 * H);
+  uint4* lo = hi + nv;
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int i = threadIdx.x + c * kNormThreads;
+    if (i < nv) {
+      float f[8], g[8], h[8], l[8];
+      unpack8(xv[c], f);
+      unpack8(wv[c], g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float n = f[j] * r * g[j];
+        h[j] = __bfloat162float(__float2bfloat16_rn(n));
+        l[j] = n - h[j];
+        amax = fmaxf(amax, fabsf(n));
+      }
+      hi[i] = pack8(h);
+      lo[i] = pack8(l);
+    }
+  }
+  if (!normed_q) return;
+  amax = block_reduce(amax, red, true);
+  const float scale = amax > 0.f ? amax / 448.f : 1.f;
+  const float inv = 1.f / scale;
+  if (threadIdx.x == 0) normed_scale[t] = scale;
+  uint2* q = reinterpret_cast<uint2*>(normed_q + size_t(t) * H);
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int i = threadIdx.x + c * kNormThreads;
+    if (i < nv) {
+      float f[8], g[8], n[8];
+      unpack8(xv[c], f);
+      unpack8(wv[c], g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) n[j] = f[j] * r * g[j] * inv;
+      q[i] = make_uint2(e4m3x4(n[0], n[1], n[2], n[3]), e4m3x4(n[4], n[5], n[6], n[7]));
+    }
+  }
+}
+
 // Split-K router, second half (one warp per token).  Lane l sums the
 // partial logits of experts l, l + 32, ... over the splits in split order
 // (all loads of a group of 8 splits in flight, each warp load one coalesced
@@ -401,9 +482,19 @@ cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* nor
                            __nv_bfloat16* residual, __nv_bfloat16* gate_a, uint8_t* normed_q,
                            float* normed_scale, int T, int H, float eps, int* hist_clear,
                            int n_clear, cudaStream_t stream) {
-  rmsnorm_kernel<<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, normed_q,
-                                                 normed_scale, H, eps, hist_clear,
-                                                 hist_clear ? n_clear : 0);
+  const int nc = hist_clear ? n_clear : 0;
+  const int chunks = (H / 8 + kNormThreads - 1) / kNormThreads;
+  if (chunks <= 2)
+    rmsnorm_reg_kernel<2><<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a,
+                                                          normed_q, normed_scale, H, eps,
+                                                          hist_clear, nc);
+  else if (chunks <= 8)
+    rmsnorm_reg_kernel<8><<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a,
+                                                          normed_q, normed_scale, H, eps,
+                                                          hist_clear, nc);
+  else
+    rmsnorm_kernel<<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, normed_q,
+                                                   normed_scale, H, eps, hist_clear, nc);
   return cudaGetLastError();
 }
 
