@@ -56,6 +56,9 @@ struct RouteParams {
 
 constexpr int kRowChunks = 16;  // 16-byte chunks per lane of one router row (H <= 4096)
 
+// MAXT: the token count rounded up to 1, 2, 4 or 8; the per-token loops are
+// unrolled to MAXT, which keeps the code of small batches short.
+template <int MAXT>
 __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
   extern __shared__ __align__(16) uint8_t dsm[];
   __shared__ float rs[kDecodeMaxT];
@@ -95,14 +98,14 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
   //    logit_e = r_t * (G_e . (x_t * w)), so the dot products need not wait
   //    for the norm
   float* xw = reinterpret_cast<float*>(dsm);  // [T][H]
-  float ss[kDecodeMaxT];
+  float ss[MAXT];
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxT; ++t) ss[t] = 0.f;
+  for (int t = 0; t < MAXT; ++t) ss[t] = 0.f;
   for (int c = threadIdx.x; c < nv; c += kThreads) {
     float g[8];
     unpack8(reinterpret_cast<const uint4*>(p.norm_w)[c], g);
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxT; ++t) {
+    for (int t = 0; t < MAXT; ++t) {
       if (t < T) {
         float f[8];
         unpack8(reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c], f);
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
     }
   }
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxT; ++t) {
+  for (int t = 0; t < MAXT; ++t) {
     const float v = warp_sum(ss[t]);
     if (lane == 0) red[warp][t] = v;
   }
@@ -131,9 +134,9 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
 
   // 3. router logits (fp32) of this warp's expert row
   if (e_row < p.E) {
-    float acc[kDecodeMaxT];
+    float acc[MAXT];
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.f;
+    for (int t = 0; t < MAXT; ++t) acc[t] = 0.f;
 #pragma unroll
     for (int c = 0; c < kRowChunks; ++c) {
       const int i = c * 256 + lane * 8;
@@ -141,7 +144,7 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
         float gf[8];
         unpack8(gv[c], gf);
 #pragma unroll
-        for (int t = 0; t < kDecodeMaxT; ++t) {
+        for (int t = 0; t < MAXT; ++t) {
           if (t < T) {
             const float4 a = *reinterpret_cast<const float4*>(xw + t * H + i);
             const float4 b = *reinterpret_cast<const float4*>(xw + t * H + i + 4);
@@ -152,7 +155,7 @@ __global__ void __launch_bounds__(kThreads) decode_route(const RouteParams p) {
       }
     }
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxT; ++t) {
+    for (int t = 0; t < MAXT; ++t) {
       if (t < T) {
         const float v = warp_sum(acc[t]);
         if (lane == 0) p.ws.logits[t * p.E + e_row] = v * rs[t];
@@ -257,7 +260,17 @@ bool decode_supported(const moe_config& c) {
 }
 
 cudaError_t prepare_decode() {
-  return cudaFuncSetAttribute(decode_route, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(decode_route<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(kMaxRouteSmem))) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(decode_route<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(kMaxRouteSmem))) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(decode_route<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(kMaxRouteSmem))) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(decode_route<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               int(kMaxRouteSmem));
 }
 
@@ -289,7 +302,10 @@ cudaError_t launch_decode_route(const DecodeRouteArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_route, rp);
+  if (a.T <= 1) return cudaLaunchKernelEx(&cfg, decode_route<1>, rp);
+  if (a.T <= 2) return cudaLaunchKernelEx(&cfg, decode_route<2>, rp);
+  if (a.T <= 4) return cudaLaunchKernelEx(&cfg, decode_route<4>, rp);
+  return cudaLaunchKernelEx(&cfg, decode_route<8>, rp);
 }
 
 }  // namespace moe

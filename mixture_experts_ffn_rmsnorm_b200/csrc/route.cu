@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(
 
 // Split-K router, second half (one warp per token).  Lane l sums the
 // partial logits of experts l, l + 32, ... over the splits in split order
-// (all loads of a group of 8 splits in flight, each warp load one coalesced
+// (two splits' loads in flight at a time, each warp load one coalesced
 // 128-byte row segment), then the warp runs the sigmoid top-k on the sums
 // and adds the token's choices to its 128-token tile's expert histogram.
 __global__ void __launch_bounds__(256) router_reduce_kernel(
@@ -222,25 +222,26 @@ __global__ void __launch_bounds__(256) router_reduce_kernel(
   const int lane = threadIdx.x & 31;
   const size_t sstride = size_t(rows_cap) * E;
   const float* src = part + size_t(t) * E + lane;
+  const int nj = (E + 31) / 32;  // experts per lane (<= 8)
   float acc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  // splits in order, two at a time so that their loads are in flight together
+  int s = 0;
+  for (; s + 2 <= ks; s += 2) {
+    float a[8], b[8];
 #pragma unroll
-  for (int s0 = 0; s0 < kRouterMaxSplit; s0 += 8) {
-    if (s0 < ks) {
-      float v[8][8];
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          v[s][j] = (s0 + s < ks && lane + 32 * j < E)
-                        ? __ldcg(src + size_t(s0 + s) * sstride + 32 * j)
-                        : 0.f;
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] += v[s][j];
+    for (int j = 0; j < 8; ++j) {
+      a[j] = j < nj && lane + 32 * j < E ? __ldcg(src + size_t(s) * sstride + 32 * j) : 0.f;
+      b[j] = j < nj && lane + 32 * j < E ? __ldcg(src + size_t(s + 1) * sstride + 32 * j) : 0.f;
     }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = (acc[j] + a[j]) + b[j];
+  }
+  if (s < ks) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      acc[j] += j < nj && lane + 32 * j < E ? __ldcg(src + size_t(s) * sstride + 32 * j) : 0.f;
   }
   const int e = warp_topk_regs(acc, bias, E, k, rsf, idx + size_t(t) * k, w + size_t(t) * k);
   // (an out-of-range id comes only from NaN logits; the sort flags it)
