@@ -1,12 +1,15 @@
 /*
  * moe_b200.h - C ABI of the B200 (sm_100a) Nemotron-H MoE FFN layer.
  *
- * The layer (NemotronMoeLayer, nemotron_moe.rs, module documentation):
- *   RMS norm, gate, sigmoid top-k routing, (fc1 if latent), routed up, relu^2
- *   and down, weighted sum, (fc2 if latent), plus the shared expert (up,
- *   relu^2, down), summed and added to `hidden`.  Routing stays on the device:
- *   nothing is read back to the host during a forward pass (same module
- *   documentation; MoeLayer, `forward`: "zero D2H").
+ * The layer (NemotronMoeLayer, nemotron_moe.rs, module documentation): the
+ * tokens are RMS-normalised and scored by the gate; a sigmoid top-k picks the
+ * routed experts of each token.  Each chosen expert applies its up projection,
+ * relu^2 and its down projection (between an fc1 into and an fc2 out of the
+ * latent width for LatentMoE), and the expert outputs are combined with the
+ * routing weights.  The always-on shared expert (up, relu^2, down) runs on the
+ * normed tokens too, and both results are added to `hidden`.  The routing
+ * never leaves the device: a forward pass copies nothing back to the host
+ * (same module documentation; MoeLayer, `forward`).
  *
  * Notation: T tokens, H hidden_size, E num_experts, k top_k, I moe_inter,
  * S shared_inter, L latent_size (0 = direct), D = (L ? L : H) the width the
@@ -114,7 +117,7 @@ typedef struct moe_handle moe_handle;
 /* Which implementation moe_forward_path runs. */
 typedef enum {
   MOE_PATH_AUTO = 0,     /* decode path for num_tokens <= MOE_DECODE_MAX_TOKENS, else prefill */
-  MOE_PATH_DECODE = 1,   /* bandwidth-bound expert GEMVs (num_tokens <= MOE_DECODE_MAX_TOKENS) */
+  MOE_PATH_DECODE = 1,   /* weight-streaming tensor-core decode, weights x tokens (num_tokens <= MOE_DECODE_MAX_TOKENS) */
   MOE_PATH_PREFILL = 2   /* sort by expert + tcgen05 grouped GEMMs (any num_tokens) */
 } moe_path;
 
@@ -128,7 +131,7 @@ typedef enum {
 MOE_API moe_status moe_create(const moe_config* config, const moe_weights* weights, moe_handle** out);
 
 /* One forward pass over num_tokens tokens, enqueued on `stream`
- * (NemotronMoeLayer `prefill` / `decode`: "modifying hidden in-place").
+ * (NemotronMoeLayer `prefill` / `decode`, which update hidden in place).
  *   hidden   [T, H] bf16, device, read then overwritten with the layer output
  *            residual_in + routed + shared (rounded once to bf16);
  *   residual [T, H] bf16, device, written with the pre-layer hidden (its

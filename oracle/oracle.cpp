@@ -7,10 +7,11 @@
 //
 // What it follows (page = "NemotronMoeLayer" rustdoc and its source
 // nemotron_moe.rs; "MoeLayer" = the generic MoE component page):
-//   * forward order: nemotron_moe.rs, module documentation ("Forward: RMS
-//     norm, gate, sigmoid top-k routing, (fc1 if latent), routed up, relu^2
-//     and down, weighted sum, (fc2 if latent), plus the shared expert (up,
-//     relu^2, down), summed and added to hidden");
+//   * forward order: nemotron_moe.rs, module documentation.  The tokens are
+//     normalised, gated and routed (sigmoid top-k); the routed experts run
+//     up, relu^2 and down (inside fc1 / fc2 when latent) and are combined
+//     with the routing weights; the shared expert (up, relu^2, down) is added,
+//     and so is the layer input;
 //   * direct vs LatentMoE shapes: same module documentation;
 //   * norm -> gate -> shared up -> fc1 order and the scaling factor:
 //     nemotron_moe.rs, `prefill`;
