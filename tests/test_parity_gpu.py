@@ -215,6 +215,43 @@ def test_host_buffer_entry_point():
     assert np.array_equal(r.numpy().view(np.uint16), inp.hidden)
 
 
+@pytest.mark.parametrize("name,T", [("tiny", 16), ("decode", 1), ("decode", 8)])
+def test_host_entry_point_repeated_calls(name, T):
+    # same buffers several times in a row (the library replays a captured
+    # sequence from the second call on), then other buffers, then pageable
+    # memory: every call gives the device path's output bit for bit
+    from workloads import bf16_to_f32
+    inp, layer, orc = setup(name, T=8, max_tokens=8) if name == "decode" else setup(name)
+    hb = inp.hidden[:T]
+    ref, _, ref_idx, _ = run_forward(layer, hb, moe.PATH_AUTO)
+    src = torch.from_numpy(hb.view(np.int16).copy())
+    h = src.clone().pin_memory()
+    r = torch.empty_like(h).pin_memory()
+    idx = torch.empty((T, layer.cfg.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, layer.cfg.top_k), dtype=torch.float32, device="cuda")
+    for _ in range(4):
+        h.copy_(src)
+        layer.forward_host(h, r)
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_to_f32(h.numpy().view(np.uint16)), ref)
+        assert np.array_equal(r.numpy().view(np.uint16), hb)
+        layer.copy_routing(idx, w)
+        torch.cuda.synchronize()
+        assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    h2 = src.clone().pin_memory()
+    for _ in range(2):
+        h2.copy_(src)
+        layer.forward_host(h2)
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_to_f32(h2.numpy().view(np.uint16)), ref)
+    hp = src.clone()  # pageable
+    for _ in range(2):
+        hp.copy_(src)
+        layer.forward_host(hp)
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_to_f32(hp.numpy().view(np.uint16)), ref)
+
+
 def test_error_codes():
     inp, layer, orc = setup("tiny")
     hid = to_dev(inp.hidden)
