@@ -64,8 +64,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         return _lib
     p = path or os.environ.get("MOE_B200_LIBRARY") or LIB_PATH
     if not os.path.exists(p):
+        if p != LIB_PATH:  # an explicit library that is not there: no substitute
+            raise FileNotFoundError(f"libmoe_b200: {p} does not exist")
         from . import build as _build
-        _build.build()
+        _build.build()  # raises when nvcc fails; there is no fallback implementation
     lib = ctypes.CDLL(p)
     V, I32 = ctypes.c_void_p, ctypes.c_int32
     sig = {

@@ -111,3 +111,22 @@ def test_static_sort_validates_on_host():
     assert lib.moe_sort_static(p, 10, 17, 64, p, p, p, None, None) == 1
     assert lib.moe_sort_static(p, 10, 4, 257, p, p, p, None, None) == 1
     assert lib.moe_sort_static(p, 10, 9, 8, p, p, p, None, None) == 1
+
+
+def test_missing_library_fails_loudly():
+    # no fallback: a library path that does not exist is an error, in a fresh
+    # interpreter (the loaded library is cached per process)
+    import subprocess
+    import sys
+    code = ("import mixture_experts_ffn_rmsnorm_b200 as m\n"
+            "try:\n"
+            "    m.load_library()\n"
+            "except FileNotFoundError as e:\n"
+            "    print('raised', e)\n"
+            "else:\n"
+            "    print('loaded')\n")
+    env = dict(os.environ, MOE_B200_LIBRARY="/nonexistent/libmoe_b200.so")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.startswith("raised"), r.stdout
