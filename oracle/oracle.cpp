@@ -18,7 +18,7 @@
 //   * sort / grouped GEMM / unpermute + weighted reduce pipeline: MoeLayer,
 //     `forward_prefill`;
 //   * top_k validation: nemotron_moe.rs, `new` and the module invariants.
-// Readings where the pages are silent (all listed in the design doc):
+// Readings where the pages are silent (each one stated here):
 //   R1 the residual buffer receives the pre-layer hidden; output =
 //      hidden + routed + shared (its input value is not read);
 //   R2 gate logits from the un-rounded normed vector;

@@ -62,8 +62,11 @@ class MoEShape:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads.  rsf / bias / latent readings where a workload is silent
-# are listed in DESIGN.md ("Readings").
+# The five workloads.  Where a workload's description is silent: rsf is 2.5
+# for the three Nemotron-H-sized direct layers (decode, prefill, skew_fp8) and
+# 1.0 for tiny and latent; the selection bias is zero unless given (uniform
+# for decode, Zipf for skew_fp8); the latent layer's shared expert works on
+# the hidden width H.
 WORKLOADS: Dict[str, MoEShape] = {
     "tiny": MoEShape("tiny", T=16, H=256, E=8, k=2, I=128, S=256, L=0,
                      rsf=1.0, bias="none", seed=0),
