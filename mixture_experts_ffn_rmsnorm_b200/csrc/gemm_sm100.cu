@@ -5,7 +5,11 @@
 // each expert's weights loaded once), run together with a dense "class" of
 // tiles in the same launch (the always-on shared expert, nemotron_moe.rs
 // `prefill`, or LatentMoE fc1 / fc2), and the router GEMM with the sigmoid
-// top-k routing fused into its epilogue.
+// top-k routing fused into its epilogue (or, with K split over idle SMs,
+// storing fp32 partial logits for the reduction kernel).  The decode launches
+// (BN = 16: weights as the 128-row operand, tokens as N) use the same kernel
+// with a stream-K schedule; the down launch accumulates all segments of a
+// 128-row output block over their concatenated K.
 //
 // Structure (one CTA per SM, persistent over a static round-robin tile list):
 //   warp 0   one lane issues TMA loads of A (128 x 128 B) and B (BN x 128 B)

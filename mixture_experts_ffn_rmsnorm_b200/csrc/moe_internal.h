@@ -22,7 +22,8 @@ enum EpiKind : int {
   EPI_TOPK = 3,        // sigmoid top-k routing of the row (gate logits never stored)
   EPI_BLEND = 4,       // out = bf16(acc + blend_s + blend_res)  (LatentMoE fc2)
   EPI_DEC_UP = 5,      // decode, weights x tokens: relu^2 (x routing weight) -> token-major rows
-  EPI_DEC_DOWN = 6,    // decode, weights x tokens: fp32 partial per segment, last arriver sums
+  EPI_DEC_DOWN = 6,    // decode, weights x tokens: fp32 partial per piece, the last piece
+                       // of a 128-row output block sums them with the residual
 };
 
 // Decode tiles multiply 128 weight rows (A) by the <= 16 token vectors (B,
