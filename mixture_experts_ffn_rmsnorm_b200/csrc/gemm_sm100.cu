@@ -9,9 +9,11 @@
 // storing fp32 partial logits for the reduction kernel).  The decode launches
 // (BN = 16: weights as the 128-row operand, tokens as N) use the same kernel
 // with a stream-K schedule; the down launch accumulates all segments of a
-// 128-row output block over their concatenated K.
+// 128-row output block over their concatenated K.  The grouped up and down
+// launches take their tiles dynamically from a device counter; the router
+// and fc2 launches walk a static round-robin.
 //
-// Structure (one CTA per SM, persistent over a static round-robin tile list):
+// Structure (one CTA per SM, persistent over its tiles):
 //   warp 0   one lane issues TMA loads of A (128 x 128 B) and B (BN x 128 B)
 //            K-blocks into a STAGES-deep shared-memory ring (128-byte swizzle);
 //   warp 1   owns TMEM (2 x BN fp32 columns = two accumulators) and one lane
@@ -40,7 +42,7 @@ struct Traits {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kKSteps = 4;                 // 4 x 32 bytes of K per stage
   static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr int kSmem = STAGES * kStageBytes + 1024 + 256;
+  static constexpr int kSmem = STAGES * kStageBytes + 1024 + 512;
   static_assert(kTmemCols == 32 || kTmemCols == 256 || kTmemCols == 512,
                 "TMEM allocation must be a power of two >= 32");
 };
@@ -223,6 +225,19 @@ __device__ __forceinline__ bool work_item(const GemmParams& p, const DecSched& d
   if (w >= W) return false;
   *t = decode_tile<BN>(p, w, W0);
   return true;
+}
+
+// Dynamic schedule: the producer publishes each tile index through a ring
+// of kTileRing slots that the MMA thread and the four epilogue warps read in
+// the same order.
+constexpr int kTileRing = 8;
+
+// Order of the dynamically handed-out tiles: the shared class (class 1,
+// whose tiles have the longer K) first, so that the short routed tiles
+// fill the end of the launch.
+__device__ __forceinline__ int dyn_tile_index(int j, int W0, int W) {
+  const int W1 = W - W0;
+  return j < W1 ? W0 + j : j - W1;
 }
 
 __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort) {
@@ -429,6 +444,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* rfull = drain + 2;  // tile-index ring (dynamic schedule)
+  uint64_t* rempty = rfull + kTileRing;
+  volatile int* ring = reinterpret_cast<volatile int*>(rempty + kTileRing);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -443,6 +461,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[b], 4);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < kTileRing; ++s) {
+      mbar_init(&rfull[s], 1);
+      mbar_init(&rempty[s], 5);  // the MMA thread and the four epilogue warps
+    }
     *abort = 0;
     fence_barrier_init();
   }
@@ -495,6 +517,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int W1 = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
     W = W0 + W1;
   }
+  const bool dyn = p.sched != nullptr && !p.dec_count;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -525,13 +548,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                       pend_x[j], pend_y[j]);
         early = false;
       };
+      // dynamic schedule: the next tile (the first is blockIdx.x) is taken
+      // from the counter two k-blocks before the current tile's last load
+      int nxt = int(blockIdx.x);
+      bool fetched = true;
       for (int it = 0; ok; ++it) {
         Tile t;
-        if (!work_item<BN>(p, ds, W, W0, it, &t)) break;
+        if (dyn) {
+          const int slot = it & (kTileRing - 1);
+          if (!mbar_wait(&rempty[slot], ((it / kTileRing) & 1) ^ 1u, abort)) {
+            record_timeout(p, abort);
+            break;
+          }
+          const int w = nxt < W ? dyn_tile_index(nxt, W0, W) : -1;
+          ring[slot] = w;
+          mbar_arrive(&rfull[slot]);
+          if (w < 0) break;
+          t = decode_tile<BN>(p, w, W0);
+          fetched = false;
+        } else if (!work_item<BN>(p, ds, W, W0, it, &t)) {
+          break;
+        }
         const GemmClass& C = p.cls[t.c];
         const int bk = stage_k(C);
         const int nk = t.k1 >= 0 ? t.k1 : (C.K + bk - 1) / bk;
+        const int fetch_kb = nk - 2 > t.k0 ? nk - 2 : t.k0;
         for (int kb = t.k0; kb < nk; ++kb) {
+          if (!fetched && kb == fetch_kb) {
+            nxt = int(gridDim.x) + atomicAdd(p.sched, 1);
+            fetched = true;
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) {
             record_timeout(p, abort);
             ok = false;
@@ -566,6 +612,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           if (early && npend == STAGES) flush_pending();
         }
+        if (ok && !fetched) {
+          nxt = int(gridDim.x) + atomicAdd(p.sched, 1);
+          fetched = true;
+        }
       }
       if (early) flush_pending();
       if (!ok) {
@@ -598,7 +648,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int it = 0; ok; ++it) {
         Tile t;
-        if (!work_item<BN>(p, ds, W, W0, it, &t)) break;
+        if (dyn) {
+          const int slot = it & (kTileRing - 1);
+          if (!mbar_wait(&rfull[slot], (it / kTileRing) & 1, abort)) {
+            record_timeout(p, abort);
+            break;
+          }
+          const int w = ring[slot];
+          mbar_arrive(&rempty[slot]);
+          if (w < 0) break;
+          t = decode_tile<BN>(p, w, W0);
+        } else if (!work_item<BN>(p, ds, W, W0, it, &t)) {
+          break;
+        }
         const bool f8 = p.cls[t.c].fp8 != 0;
         const int bk = f8 ? 128 : 64;
         const int nk = t.k1 >= 0 ? t.k1 : (p.cls[t.c].K + bk - 1) / bk;
@@ -648,7 +710,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int rloc = q * 32 + lane;
     for (int it = 0;; ++it) {
       Tile t;
-      if (!work_item<BN>(p, ds, W, W0, it, &t)) break;
+      if (dyn) {  // lane 0 takes the index from the ring for the warp
+        const int slot = it & (kTileRing - 1);
+        int w = -1, got = 1;
+        if (lane == 0) {
+          got = mbar_wait(&rfull[slot], (it / kTileRing) & 1, abort);
+          if (got) {
+            w = ring[slot];
+            mbar_arrive(&rempty[slot]);
+          } else {
+            record_timeout(p, abort);
+          }
+        }
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!__shfl_sync(0xffffffffu, got, 0) || w < 0) break;
+        t = decode_tile<BN>(p, w, W0);
+      } else if (!work_item<BN>(p, ds, W, W0, it, &t)) {
+        break;
+      }
       const GemmClass& C = p.cls[t.c];
       const int ab = it & 1;
       const uint32_t aph = (it >> 1) & 1;
@@ -750,6 +829,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Tr::kTmemCols);
+  }
+  if (dyn && threadIdx.x == 0) {
+    // every producer of the grid has taken its last index once all CTAs
+    // have counted themselves out: the last one zeroes the counters
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1) == int(gridDim.x) - 1) {
+      atomicExch(p.sched, 0);
+      atomicExch(p.sched + 1, 0);
+    }
   }
 }
 

@@ -101,6 +101,7 @@ struct moe_handle {
   int32_t* expert_hist;    // [ceil(Tm/128), E]
   int32_t* n_mtiles;
   int32_t* status;
+  int32_t* sched;  // [4] dynamic tile schedule counters of the up and down launches
   int32_t* perm;   // [Rm]
   int32_t* inv;    // [Rm]
   bf16* z;         // [Tm, L]   latent fc1 output
@@ -201,6 +202,7 @@ void carve(moe_handle* h, char* base) {
   h->expert_hist = cv.take<int32_t>((Tm + moe::kBM - 1) / moe::kBM * E);
   h->n_mtiles = cv.take<int32_t>(1);
   h->status = cv.take<int32_t>(1);
+  h->sched = cv.take<int32_t>(4);
   h->perm = cv.take<int32_t>(Rm);
   h->inv = cv.take<int32_t>(Rm);
   h->z = L ? cv.take<bf16>(Tm * L) : nullptr;
@@ -401,6 +403,7 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.n_mtiles = h->n_mtiles;
   p.group_off = h->off;
   p.status = h->status;
+  p.sched = h->sched;
   MOE_TRY(moe::launch_grouped_gemm(p, h->up_bn, h->num_sms, st));
   log->done(st);
 
@@ -421,6 +424,7 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.tmA[1] = h->tm_sdown_a;
   p.tmB[1] = h->tm_sdown_w;
   p.cls[1] = dense_class(S, H, T, moe::EPI_F32, h->s, H, h->down_bn);
+  p.sched = h->sched + 2;
   MOE_TRY(moe::launch_grouped_gemm(p, h->down_bn, h->num_sms, st));
   log->done(st);
 

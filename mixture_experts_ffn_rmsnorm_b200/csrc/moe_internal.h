@@ -149,6 +149,12 @@ struct GemmParams {
   const void* l2_prefetch[2];
   size_t l2_prefetch_bytes[2];
   DecodeEpilogue dec;
+  // Dynamic tile schedule (non-decode launches; null = static round-robin):
+  // sched[0] hands out tile indices past the first gridDim.x, sched[1]
+  // counts exiting CTAs.  Both are zero before the launch and the last CTA
+  // to exit zeroes them again.  Tiles are then taken shared class first
+  // (its tiles have the longer K), routed class after.
+  int* sched;
 };
 
 // Launch the persistent grouped GEMM (bn = 16, 128 or 256); the operand type
