@@ -320,12 +320,13 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
     const int nk = (2 * c.hidden_size + 63) / 64;
     const int other = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
     ks = h->num_sms > other ? (h->num_sms - other) / mt : 1;
-    if (other >= h->num_sms) {
-      // The other class alone fills the SMs (LatentMoE fc1): cut the router
-      // tiles (K = 2H) into pieces of half the other class's K, so that no
-      // router tile is the launch's long pole.
+    if (other > 0) {
+      // With LatentMoE fc1 in the launch, cut the router tiles (K = 2H) into
+      // pieces of at most half fc1's K, so that no router tile is the
+      // launch's long pole (more pieces when idle SMs allow).
       const int nko = (p.cls[1].K + 63) / 64;
-      ks = 2 * ((nk + nko - 1) / nko);
+      const int cut = 2 * ((nk + nko - 1) / nko);
+      if (ks < cut) ks = cut;
     }
     if (ks > h->num_sms / mt) ks = h->num_sms / mt;  // capacity of the partial logits
     ks = ks < 1 ? 1 : (ks > moe::kRouterMaxSplit ? moe::kRouterMaxSplit : ks);
