@@ -206,21 +206,31 @@ def test_sort_bit_exact(name, T, skew):
 
 # --------------------------------------------------------- API behaviour ---
 
-def test_graph_capture_and_replay():
-    # no host sync, allocation or D2H inside the forward: it captures
-    inp, layer, orc = setup("tiny")
-    ref = run_forward(layer, inp.hidden, moe.PATH_PREFILL)[0]
-    hid = to_dev(inp.hidden)
+@pytest.mark.parametrize("name,T,path", [("tiny", 16, moe.PATH_PREFILL),
+                                         ("decode", 1, moe.PATH_DECODE),
+                                         ("decode", 8, moe.PATH_DECODE)])
+def test_graph_capture_and_replay(name, T, path):
+    # No host sync, allocation or D2H inside the forward: it captures, and a
+    # replay gives the eager call's output bit for bit.  The decode cases are
+    # the launch configuration the benchmark times (programmatic dependent
+    # launches inside a graph).
+    from workloads import bf16_to_f32
+    inp, layer, orc = setup(name, T=8, max_tokens=8) if name == "decode" else setup(name)
+    hb = inp.hidden[:T]
+    ref = run_forward(layer, hb, path)[0]
+    hid = to_dev(hb)
     res = torch.empty_like(hid)
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        layer.forward(hid, res, path=moe.PATH_PREFILL, stream=s)
-    hid.copy_(to_dev(inp.hidden))
+        layer.forward(hid, res, path=path, stream=s)
+    hid.copy_(to_dev(hb))
     g.replay()
     torch.cuda.synchronize()
-    from workloads import bf16_to_f32
     assert np.array_equal(bf16_to_f32(hid.cpu().numpy().view(np.uint16)), ref)
+    assert np.array_equal(res.cpu().numpy().view(np.uint16), hb)
+    assert layer.device_status() == 0
 
 
 def test_host_buffer_entry_point():
@@ -237,8 +247,7 @@ def test_host_buffer_entry_point():
 
 @pytest.mark.parametrize("name,T", [("tiny", 16), ("decode", 1), ("decode", 8)])
 def test_host_entry_point_repeated_calls(name, T):
-    # same buffers several times in a row (the library replays a captured
-    # sequence from the second call on), then other buffers, then pageable
+    # same buffers several times in a row, then other buffers, then pageable
     # memory: every call gives the device path's output bit for bit
     from workloads import bf16_to_f32
     inp, layer, orc = setup(name, T=8, max_tokens=8) if name == "decode" else setup(name)
