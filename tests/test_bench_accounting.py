@@ -1,0 +1,134 @@
+"""bench.py's work model on CPU: the algorithmic bytes and flops it divides
+by each kernel's time, against closed forms written out here from the
+layer's shapes, and the committed DRAM captures against that model.
+
+The closed forms count what the layer must move or compute once: every
+touched expert's weights, the shared expert, the gate, and the token rows
+(NemotronMoeLayer `prefill` / `decode`; grouped GEMM loading each expert's
+weights once, MoeLayer `forward_prefill`).
+"""
+import json
+import os
+
+import pytest
+
+import bench
+from workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _sum(stages, i):
+    return sum(st[i] for st in stages)
+
+
+def test_decode_T1_bytes_match_the_weight_stream():
+    s = WORKLOADS["decode"]
+    H, E, k, I, S = s.H, s.E, s.k, s.I, s.S
+    U, T = k, 1  # one token touches k distinct experts
+    weights = U * 2 * H * I * 2 + 2 * H * S * 2 + E * H * 2
+    tokens = H * 2 + 3 * T * H * 2
+    closed = weights + tokens
+    assert closed == 160_355_328  # 160.4 MB: a 24.5 us roofline at 6.53 TB/s
+    model = bench.stage_model(s, T, "decode", U)
+    assert [m[0] for m in model] == ["decode_route", "decode_up_gemm", "decode_down_gemm"]
+    # the model adds the intermediate activations (R x I, T x S) both ways
+    assert _sum(model, 1) == pytest.approx(closed, rel=1e-3)
+    up, down = model[1], model[2]
+    assert up[1] - (U * I * H * 2 + S * H * 2) < 64 * 1024
+    assert down[1] - (U * H * I * 2 + H * S * 2) < 64 * 1024
+
+
+@pytest.mark.parametrize("name,T,gflop", [
+    ("prefill", 1024, 164.2),   # 48 rows per expert: HBM-bound
+    ("latent", 4096, 794.6),    # tensor-bound
+])
+def test_prefill_flops_closed_form(name, T, gflop):
+    s = WORKLOADS[name]
+    H, E, k, I, S, L, D = s.H, s.E, s.k, s.I, s.S, s.L, s.D
+    R = T * k
+    closed = 2 * T * H * E + 4 * R * D * I + 4 * T * H * S + 4 * T * H * L
+    assert closed / 1e9 == pytest.approx(gflop, abs=0.05)
+    for split in (False, True):
+        model = bench.stage_model(s, T, "prefill", E, router_split=split)
+        assert _sum(model, 2) == closed
+
+
+def test_skew_fp8_splits_fp8_and_bf16_work():
+    s = WORKLOADS["skew_fp8"]
+    T = 8192
+    H, E, k, I, S = s.H, s.E, s.k, s.I, s.S
+    R = T * k
+    fp8 = 4 * R * H * I
+    bf16 = 2 * T * H * E + 4 * T * H * S
+    assert fp8 / 1e9 == pytest.approx(980.9, abs=0.05)
+    assert bf16 / 1e9 == pytest.approx(332.6, abs=0.05)
+    model = bench.stage_model(s, T, "prefill", E, router_split=True)
+    assert _sum(model, 2) == fp8 + bf16
+    names = [m[0] for m in model]
+    assert "quantize_rows" in names and "combine" in names
+    # FP8 expert weights stream one byte per element plus one fp32 scale per row
+    up = dict((m[0], m) for m in model)["grouped_up_gemm"]
+    assert up[1] >= E * I * H * 1 + E * I * 4 + S * H * 2
+
+
+def test_prefill_T1024_weight_bytes():
+    s = WORKLOADS["prefill"]
+    H, E, I, S = s.H, s.E, s.I, s.S
+    weights = E * 2 * H * I * 2 + 2 * H * S * 2 + E * H * 2
+    assert weights / 1e9 == pytest.approx(2.595, abs=0.001)
+    model = bench.stage_model(s, 1024, "prefill", E, router_split=True)
+    gemms = [m for m in model if "gemm" in m[0]]
+    assert _sum(gemms, 1) > weights
+    assert _sum(gemms, 1) < weights * 1.1
+
+
+def test_roofline_picks_the_binding_bound():
+    peaks = {"hbm_gbs": 6530.0, "bf16_tflops": 1626.0, "bf16_tflops_sustained": 1399.0,
+             "source": "measured"}
+    # 80 MB in 30 us: HBM-bound, 2.67 TB/s
+    r = bench.roofline_of("decode_down_gemm", 80e6, 1e6, 0.030, peaks, False)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(80e6 / 30e-6 / 1e9, rel=1e-3)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6530.0, rel=1e-3)
+    # 800 GFLOP in 1 ms over 1.6 GB: tensor-bound; FP8 GEMMs get twice the peak
+    r = bench.roofline_of("grouped_up_gemm", 1.6e9, 800e9, 1.0, peaks, False)
+    assert r["bound"] == "tensor" and r["peak"] == 1626.0
+    r8 = bench.roofline_of("grouped_up_gemm", 1.6e9, 800e9, 1.0, peaks, True)
+    assert r8["peak"] == 2 * 1626.0 and r8["frac"] == pytest.approx(r["frac"] / 2, rel=1e-3)
+    # non-GEMM kernels never take the FP8 factor
+    r = bench.roofline_of("combine", 1e8, 0, 0.02, peaks, True)
+    assert r["bound"] == "hbm"
+
+
+def test_committed_dram_captures_are_close_to_the_model():
+    """Every capture in profiles/traffic.json moves within 10 % of the
+    algorithmic bytes the benchmark divides by: no wasted re-reads."""
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)["kernels"]
+    assert recs
+    for key, rec in recs.items():
+        stage, workload = key.split("@")
+        name, tok = workload.split(" T=")
+        T = int(tok)
+        s = WORKLOADS[name]
+        path = "decode" if name == "decode" else "prefill"
+        U = s.k * T if path == "decode" else s.E  # T=1 decode: k experts; prefill: all
+        model = dict((m[0], m) for m in bench.stage_model(s, T, path, U, router_split=True))
+        stage_bytes = model[stage][1] if stage in model else model[stage.replace("_gemm", "_gemm_topk")][1]
+        got = rec["dram_bytes_per_launch"]
+        assert abs(got - stage_bytes) <= 0.10 * stage_bytes, (key, got, stage_bytes)
+        assert rec["capture"].startswith("profiles/") and os.path.exists(
+            os.path.join(ROOT, rec["capture"]))
+
+
+def test_sources_hash_is_stable_and_detects_change(tmp_path):
+    a = tmp_path / "a.cu"
+    a.write_text("x")
+    rel = os.path.relpath(a, bench.ROOT)
+    h1 = bench.sources_hash([rel])
+    assert h1 == bench.sources_hash([rel]) and len(h1) == 16
+    a.write_text("y")
+    assert bench.sources_hash([rel]) != h1
+    assert bench.sources_hash(["no/such/file.cu"]) is None
+    assert bench.kernel_traffic("no_such_stage", "decode T=1") is None
