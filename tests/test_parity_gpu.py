@@ -208,12 +208,14 @@ def test_sort_bit_exact(name, T, skew):
 
 @pytest.mark.parametrize("name,T,path", [("tiny", 16, moe.PATH_PREFILL),
                                          ("decode", 1, moe.PATH_DECODE),
-                                         ("decode", 8, moe.PATH_DECODE)])
+                                         ("decode", 8, moe.PATH_DECODE),
+                                         ("prefill", 1024, moe.PATH_PREFILL)])
 def test_graph_capture_and_replay(name, T, path):
     # No host sync, allocation or D2H inside the forward: it captures, and a
-    # replay gives the eager call's output bit for bit.  The decode cases are
-    # the launch configuration the benchmark times (programmatic dependent
-    # launches inside a graph).
+    # replay gives the eager call's output bit for bit.  The decode and
+    # prefill cases are the launch configuration the benchmark times (graph
+    # replay; programmatic dependent launches and device-side tile counters
+    # inside the graph).
     from workloads import bf16_to_f32
     inp, layer, orc = setup(name, T=8, max_tokens=8) if name == "decode" else setup(name)
     hb = inp.hidden[:T]
