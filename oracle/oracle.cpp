@@ -90,12 +90,23 @@ double e4m3(uint8_t b) {
   return sign ? -v : v;
 }
 
+// The 256 E4M3 values, each computed once (when the library loads) by
+// e4m3() above: looking a byte up here gives exactly e4m3(byte), without its
+// per-call ldexp.
+struct E4M3Table {
+  double v[256];
+  E4M3Table() {
+    for (int b = 0; b < 256; ++b) v[b] = e4m3(uint8_t(b));
+  }
+};
+const E4M3Table kE4M3;
+
 // Element (e, r, c) of a routed expert stack [E, rows, cols], dequantised.
 double expert_w(const oracle_cfg& c, const void* w, const float* scale,
                 int e, int r, int rows, int col, int cols) {
   size_t i = (size_t(e) * rows + r) * size_t(cols) + col;
   if (c.expert_fp8)
-    return e4m3(static_cast<const uint8_t*>(w)[i]) * double(scale[size_t(e) * rows + r]);
+    return kE4M3.v[static_cast<const uint8_t*>(w)[i]] * double(scale[size_t(e) * rows + r]);
   return bf16(static_cast<const uint16_t*>(w)[i]);
 }
 
