@@ -33,7 +33,10 @@
  *
  * Errors: every entry point validates its arguments on the host before any
  * launch and returns a moe_status; nothing is enqueued when it fails.  Launch
- * failures come back as MOE_ERR_CUDA.  Device-side bounded waits that time out
+ * failures come back as MOE_ERR_CUDA.  A handle belongs to the device that
+ * was current at moe_create: every call that takes a handle (except
+ * moe_destroy, which switches to that device itself) returns MOE_ERR_DEVICE
+ * when another device is current.  Device-side bounded waits that time out
  * set a device status word, read by moe_get_device_status.
  */
 #ifndef MOE_B200_H
@@ -59,7 +62,7 @@ typedef enum {
   MOE_ERR_TOKENS_OUT_OF_RANGE = 4, /* num_tokens outside [1, max_tokens] */
   MOE_ERR_OUT_OF_MEMORY = 5,       /* workspace allocation failed in moe_create */
   MOE_ERR_CUDA = 6,                /* a CUDA runtime call or launch failed */
-  MOE_ERR_DEVICE = 7,              /* no sm_100 device is current */
+  MOE_ERR_DEVICE = 7,              /* no sm_100 device is current, or not the handle's */
   MOE_ERR_INVALID_HANDLE = 8       /* NULL or destroyed handle */
 } moe_status;
 
@@ -200,7 +203,10 @@ MOE_API moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_token
  *   R = num_tokens * top_k): as moe_sort.
  *   status: optional device int32; set to 0, then bit 2 is OR-ed in if an
  *   id lies outside [0, num_experts) (that row is skipped).  NULL uses a
- *   word in the scratch.
+ *   word in the scratch that the caller cannot read: a bad id then goes
+ *   unreported, and the entries of perm and inv it would have filled
+ *   (perm[off[E]..R) and inv of its row) are left unwritten.  Pass a status
+ *   word unless the ids are known to be in range.
  *   stream: cudaStream_t (NULL = legacy default stream).
  *
  * Errors (nothing is launched): MOE_ERR_NULL_POINTER for a NULL idx, perm,
@@ -212,7 +218,9 @@ MOE_API moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_token
  *
  * The first call on a device does set-up (it looks up the scratch array's
  * device address, which may load the module on that device); make it before
- * any stream capture.  The scratch is shared by all calls on a device, so
+ * any stream capture.  The address is kept for the device's primary context
+ * (the runtime's context): call it with that context current, and not after
+ * cudaDeviceReset, which discards the context the address belongs to.  The scratch is shared by all calls on a device, so
  * calls that overlap in time there (other streams or host threads) race;
  * the caller serialises them. */
 MOE_API moe_status moe_sort_static(const int32_t* idx, int32_t num_tokens, int32_t top_k,
@@ -224,6 +232,15 @@ MOE_API moe_status moe_sort_static(const int32_t* idx, int32_t num_tokens, int32
  * meaning as moe_route's outputs); num_tokens must equal that call's. */
 MOE_API moe_status moe_copy_routing(moe_handle* h, int32_t* idx, float* w, int32_t num_tokens,
                                     void* stream);
+
+/* Copy the sort by expert used by the last moe_forward* call on this handle
+ * (prefill path) into perm [R], inv [R] and off [E+1] int32 (device
+ * pointers, R = num_tokens * top_k; same meaning as moe_sort's outputs, for
+ * the routing moe_copy_routing returns).  num_tokens must equal that call's.
+ * MOE_ERR_INVALID_CONFIG when that call took the decode path, which groups
+ * tokens by expert without a sort. */
+MOE_API moe_status moe_copy_sort(moe_handle* h, int32_t* perm, int32_t* inv, int32_t* off,
+                                 int32_t num_tokens, void* stream);
 
 /* Copy the device status word into *status (0 = no device-side timeout) and
  * clear it.  Synchronises the stream (debug use only). */
@@ -238,6 +255,10 @@ MOE_API moe_status moe_set_stage_events(moe_handle* h, void* const* events, int3
 
 /* Number of kernel launches the last moe_forward* call enqueued. */
 MOE_API int32_t moe_last_launch_count(const moe_handle* h);
+
+/* Path the last moe_forward* call took: MOE_PATH_DECODE or MOE_PATH_PREFILL
+ * (-1 for an invalid handle or before the first forward). */
+MOE_API int32_t moe_last_path(const moe_handle* h);
 
 #ifdef __cplusplus
 }

@@ -27,7 +27,8 @@ WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
 EXPORTED_SYMBOLS = ("moe_create", "moe_forward", "moe_forward_path", "moe_forward_host",
                     "moe_destroy", "moe_status_string", "moe_route", "moe_sort",
                     "moe_get_device_status", "moe_last_launch_count", "moe_copy_routing",
-                    "moe_set_stage_events", "moe_sort_static")
+                    "moe_set_stage_events", "moe_sort_static", "moe_copy_sort",
+                    "moe_last_path")
 
 
 class MoEError(RuntimeError):
@@ -84,6 +85,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_copy_routing": ([V, V, V, I32, V], ctypes.c_int),
         "moe_set_stage_events": ([V, V, I32], ctypes.c_int),
         "moe_sort_static": ([V, I32, I32, I32, V, V, V, V, V], ctypes.c_int),
+        "moe_copy_sort": ([V, V, V, V, I32, V], ctypes.c_int),
+        "moe_last_path": ([V], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -172,6 +175,12 @@ class MoELayer:
         self._check(self.lib.moe_copy_routing(self.handle, _ptr(idx), _ptr(w), idx.shape[0],
                                               _stream_ptr(stream)), "moe_copy_routing")
 
+    def copy_sort(self, perm, inv, off, num_tokens, stream=None):
+        """Sort by expert (perm [R], inv [R], off [E+1]) of the last forward
+        (prefill path); int32 tensors on the device."""
+        self._check(self.lib.moe_copy_sort(self.handle, _ptr(perm), _ptr(inv), _ptr(off),
+                                           num_tokens, _stream_ptr(stream)), "moe_copy_sort")
+
     def device_status(self, stream=None) -> int:
         v = ctypes.c_int32(0)
         self._check(self.lib.moe_get_device_status(self.handle, ctypes.byref(v),
@@ -193,6 +202,10 @@ class MoELayer:
 
     def last_launch_count(self) -> int:
         return int(self.lib.moe_last_launch_count(self.handle))
+
+    def last_path_decode(self) -> bool:
+        """Whether the last forward took the decode path."""
+        return int(self.lib.moe_last_path(self.handle)) == PATH_DECODE
 
     def close(self):
         if self.handle:

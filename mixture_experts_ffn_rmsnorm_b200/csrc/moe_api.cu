@@ -139,6 +139,17 @@ moe_status check_handle(const moe_handle* h) {
   return (h && h->magic == kMagic) ? MOE_OK : MOE_ERR_INVALID_HANDLE;
 }
 
+// A valid handle whose device is the current one: its workspace, weights
+// and tensor maps live on that device, so a call made while another device
+// is current is refused before anything is enqueued.
+moe_status check_handle_device(const moe_handle* h) {
+  moe_status st = check_handle(h);
+  if (st != MOE_OK) return st;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) return MOE_ERR_DEVICE;
+  return MOE_OK;
+}
+
 moe_status validate_config(const moe_config* c) {
   if (c->hidden_size <= 0 || c->num_experts <= 0 || c->moe_inter <= 0 || c->shared_inter <= 0 ||
       c->latent_size < 0 || c->max_tokens < 1)
@@ -602,7 +613,7 @@ moe_status moe_destroy(moe_handle* h) {
 
 moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t num_tokens,
                             int32_t path, void* stream) {
-  moe_status st = check_handle(h);
+  moe_status st = check_handle_device(h);
   if (st != MOE_OK) return st;
   if (!hidden || !residual) return MOE_ERR_NULL_POINTER;
   if (!aligned16(hidden) || !aligned16(residual)) return MOE_ERR_MISALIGNED;
@@ -639,7 +650,7 @@ moe_status moe_forward(moe_handle* h, void* hidden, void* residual, int32_t num_
 
 moe_status moe_forward_host(moe_handle* h, void* hidden_host, void* residual_host,
                             int32_t num_tokens, void* stream) {
-  moe_status st = check_handle(h);
+  moe_status st = check_handle_device(h);
   if (st != MOE_OK) return st;
   if (!hidden_host) return MOE_ERR_NULL_POINTER;
   if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
@@ -656,7 +667,7 @@ moe_status moe_forward_host(moe_handle* h, void* hidden_host, void* residual_hos
 
 moe_status moe_route(moe_handle* h, const void* hidden, int32_t num_tokens, int32_t* idx,
                      float* w, void* stream) {
-  moe_status st = check_handle(h);
+  moe_status st = check_handle_device(h);
   if (st != MOE_OK) return st;
   if (!hidden || !idx || !w) return MOE_ERR_NULL_POINTER;
   if (!aligned16(hidden)) return MOE_ERR_MISALIGNED;
@@ -675,7 +686,7 @@ moe_status moe_route(moe_handle* h, const void* hidden, int32_t num_tokens, int3
 
 moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_tokens, int32_t* perm,
                     int32_t* inv, int32_t* off, void* stream) {
-  moe_status st = check_handle(h);
+  moe_status st = check_handle_device(h);
   if (st != MOE_OK) return st;
   if (!idx || !perm || !inv || !off) return MOE_ERR_NULL_POINTER;
   if (num_tokens < 1 || num_tokens > h->cfg.max_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
@@ -690,7 +701,7 @@ moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_tokens, int32
 
 moe_status moe_copy_routing(moe_handle* h, int32_t* idx, float* w, int32_t num_tokens,
                             void* stream) {
-  moe_status st = check_handle(h);
+  moe_status st = check_handle_device(h);
   if (st != MOE_OK) return st;
   if (!idx || !w) return MOE_ERR_NULL_POINTER;
   if (num_tokens < 1 || num_tokens != h->last_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
@@ -703,8 +714,24 @@ moe_status moe_copy_routing(moe_handle* h, int32_t* idx, float* w, int32_t num_t
   return MOE_OK;
 }
 
+moe_status moe_copy_sort(moe_handle* h, int32_t* perm, int32_t* inv, int32_t* off,
+                         int32_t num_tokens, void* stream) {
+  moe_status st = check_handle_device(h);
+  if (st != MOE_OK) return st;
+  if (!perm || !inv || !off) return MOE_ERR_NULL_POINTER;
+  if (num_tokens < 1 || num_tokens != h->last_tokens) return MOE_ERR_TOKENS_OUT_OF_RANGE;
+  if (h->last_decode) return MOE_ERR_INVALID_CONFIG;  // the decode path does not sort
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t R = size_t(num_tokens) * h->cfg.top_k;
+  MOE_TRY(cudaMemcpyAsync(perm, h->perm, R * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  MOE_TRY(cudaMemcpyAsync(inv, h->inv, R * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  MOE_TRY(cudaMemcpyAsync(off, h->off, (h->cfg.num_experts + 1) * sizeof(int32_t),
+                          cudaMemcpyDeviceToDevice, s));
+  return MOE_OK;
+}
+
 moe_status moe_get_device_status(moe_handle* h, int32_t* status, void* stream) {
-  moe_status st = check_handle(h);
+  moe_status st = check_handle_device(h);
   if (st != MOE_OK) return st;
   if (!status) return MOE_ERR_NULL_POINTER;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -725,6 +752,11 @@ moe_status moe_set_stage_events(moe_handle* h, void* const* events, int32_t coun
 
 int32_t moe_last_launch_count(const moe_handle* h) {
   return check_handle(h) == MOE_OK ? h->last_launches : -1;
+}
+
+int32_t moe_last_path(const moe_handle* h) {
+  if (check_handle(h) != MOE_OK || h->last_tokens < 1) return -1;
+  return h->last_decode ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
 }
 
 }  // extern "C"

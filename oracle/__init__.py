@@ -5,7 +5,7 @@ benchmark's CPU-baseline leg are the only users.  The CUDA library and its
 Python binding never import this package.
 
 Parity status of each function (pins in tests/test_oracle_pins.py):
-  rmsnorm, gate_logits, route, sort, forward - pinned (closed forms,
+  rmsnorm, gate_logits, route, route_weights, sort, forward - pinned (closed forms,
   brute-force enumeration, hand-computed cases, invariants).
 """
 from __future__ import annotations
@@ -55,6 +55,7 @@ def _L():
             "oracle_rmsnorm": [P, P, P, ctypes.c_int32, P],
             "oracle_gate_logits": [P, P, P, ctypes.c_int32, P, ctypes.c_int32],
             "oracle_route": [P, P, P, ctypes.c_int32, P, P, P],
+            "oracle_route_forced": [P, P, P, ctypes.c_int32, P],
             "oracle_sort": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P],
             "oracle_forward": [P, P, P, ctypes.c_int32, P, P, P, P, ctypes.c_int32],
         }.items():
@@ -145,6 +146,18 @@ class Oracle:
         assert _L().oracle_route(ctypes.byref(self.cfg), _ptr(lg), _ptr(b), T, _ptr(idx),
                                  _ptr(w), _ptr(keys)) == 0
         return idx, w, keys
+
+    def route_weights(self, logits, forced_idx) -> np.ndarray:
+        """Routing weights [T,k] f64 of the given expert sets (slot order
+        kept): rsf * sigmoid(logit_e) / sum over the set."""
+        lg = np.ascontiguousarray(logits, dtype=np.float64)
+        T = lg.shape[0]
+        f = np.ascontiguousarray(forced_idx, dtype=np.int32)
+        assert f.shape == (T, self.shape.k)
+        w = np.empty((T, self.shape.k), dtype=np.float64)
+        rc = _L().oracle_route_forced(ctypes.byref(self.cfg), _ptr(lg), _ptr(f), T, _ptr(w))
+        assert rc == 0, "oracle_route_forced rejected its arguments"
+        return w
 
     def forward(self, hidden, forced_idx=None, nthreads: int = 0):
         """(out [T,H] f64, idx [T,k] int32, weights [T,k] f64)."""

@@ -280,6 +280,21 @@ int oracle_route(const oracle_cfg* c, const double* logits, const float* bias, i
   return 0;
 }
 
+// Weights of given expert sets: forced [T,k] takes the place of the top-k
+// choice (slot order kept), wts [T,k] = rsf * s_e / sum of the set's s_e.
+int oracle_route_forced(const oracle_cfg* c, const double* logits, const int32_t* forced,
+                        int32_t T, double* wts) {
+  if (check_cfg(c) || T < 0 || !forced) return 1;
+  std::vector<int32_t> idx(c->k);
+  for (int t = 0; t < T; ++t) {
+    for (int j = 0; j < c->k; ++j)
+      if (forced[size_t(t) * c->k + j] < 0 || forced[size_t(t) * c->k + j] >= c->E) return 1;
+    route(*c, logits + size_t(t) * c->E, nullptr, forced + size_t(t) * c->k, idx.data(),
+          wts + size_t(t) * c->k, nullptr);
+  }
+  return 0;
+}
+
 // Sort the R = T*k routed rows by expert (counting sort, stable in row
 // order f = t*k + j): perm[pos] = f, inv[f] = pos, off[E+1] exclusive prefix
 // of the per-expert counts.  Returns 1 on an expert id outside [0, E).

@@ -380,3 +380,21 @@ def test_forced_routing_recomputes_weights_from_scores():
     np.testing.assert_array_equal(idx, forced)
     s = 1.0 / (1.0 + np.exp(-np.take_along_axis(lg, forced, axis=1)))
     np.testing.assert_allclose(w, 2.0 * s / s.sum(axis=1, keepdims=True), rtol=1e-14)
+
+
+def test_route_weights_of_forced_sets_match_the_scores():
+    # the weights of a given expert set: rsf * sigmoid(logit_e) / sum over
+    # the set, in the set's own slot order; forward with the same forced
+    # sets reports the same weights
+    d = _tiny(T=4, rsf=2.5)
+    o = oracle.Oracle(d)
+    lg = o.gate_logits(d.hidden)
+    forced = np.array([[6, 2], [1, 0], [7, 3], [4, 5]], dtype=np.int32)
+    w = o.route_weights(lg, forced)
+    s = 1.0 / (1.0 + np.exp(-np.take_along_axis(lg, forced, axis=1)))
+    np.testing.assert_allclose(w, 2.5 * s / s.sum(axis=1, keepdims=True), rtol=1e-14)
+    _, _, fw = o.forward(d.hidden, forced_idx=forced)
+    np.testing.assert_array_equal(w, fw)
+    # the oracle's own choice gives its own weights
+    idx, ow, _ = o.route(lg)
+    np.testing.assert_array_equal(o.route_weights(lg, idx), ow)
