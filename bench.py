@@ -65,7 +65,10 @@ def stage_model(s, T, path, U, router_split=False):
 
     U = distinct routed experts of the step (weights touched once each).
     Weight bytes use the storage width (2 for BF16, 1 for FP8 + scales).
-    Returns a list of (name, bytes, flops) in launch order.
+    Returns a list of (name, bytes, flops, fp8_flops) in launch order:
+    `flops` counts all of a kernel's multiply-adds (x2), `fp8_flops` the part
+    of them that runs on E4M3 operands (the routed experts when their weights
+    are FP8; the gate, the shared expert and fc1/fc2 are BF16).
     """
     H, E, k, I, S, L = s.H, s.E, s.k, s.I, s.S, s.L
     D = s.D
@@ -73,55 +76,79 @@ def stage_model(s, T, path, U, router_split=False):
     wb = 1 if s.expert_fp8 else 2
     up_w = U * I * D * wb + (U * I * 4 if s.expert_fp8 else 0)
     down_w = U * D * I * wb + (U * D * 4 if s.expert_fp8 else 0)
+    f8 = 1 if s.expert_fp8 else 0
     if path == "decode":
         return [
-            ("decode_route", E * H * 2 + 3 * T * H * 2 + T * E * 4, 2 * T * H * E),
+            ("decode_route", E * H * 2 + 3 * T * H * 2 + T * E * 4, 2 * T * H * E, 0),
             ("decode_up_gemm", up_w + S * H * 2 + T * H * 2 + R * I * 2 + T * S * 2,
-             2 * R * D * I + 2 * T * H * S),
+             2 * R * D * I + 2 * T * H * S, f8 * 2 * R * D * I),
             ("decode_down_gemm", down_w + H * S * 2 + R * I * 2 + T * S * 2 + T * H * 2 * 2,
-             2 * R * I * D + 2 * T * S * H),
+             2 * R * I * D + 2 * T * S * H, f8 * 2 * R * I * D),
         ]
-    st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2 + (T * H if s.expert_fp8 else 0), 0)]
+    st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2 + (T * H if s.expert_fp8 else 0), 0, 0)]
     # With split K (few token tiles) the router GEMM stores partial logits
     # and a second kernel sums them and selects; its algorithmic bytes are
     # the routing table it writes (the partials are the split's overhead).
     sel = "" if router_split else "_topk"
     if L:
         st.append((f"router_gemm{sel}+fc1", E * H * 2 + T * 2 * H * 2 + L * H * 2 + T * L * 2,
-                   2 * T * E * H + 2 * T * H * L))
+                   2 * T * E * H + 2 * T * H * L, 0))
     else:
         st.append((f"router_gemm{sel}", E * H * 2 + T * 2 * H * 2 + (0 if router_split else R * 8),
-                   2 * T * E * H))
+                   2 * T * E * H, 0))
     if router_split:
-        st.append(("router_reduce_topk", R * 8, 0))
+        st.append(("router_reduce_topk", R * 8, 0, 0))
     st += [
-        ("sort", R * 4 * 3 + (E + 1) * 4, 0),
-        ("gather", 2 * R * D * wb, 0),
+        ("sort", R * 4 * 3 + (E + 1) * 4, 0, 0),
+        # each token row is read once from HBM (its k copies come from L2)
+        # and written once per routed slot
+        ("gather", T * D * wb + R * D * wb + R * 4, 0, 0),
         ("grouped_up_gemm", up_w + S * H * 2 + R * D * wb + T * H * 2 + R * I * 2 + T * S * 2,
-         2 * R * D * I + 2 * T * H * S),
+         2 * R * D * I + 2 * T * H * S, f8 * 2 * R * D * I),
     ]
     if s.expert_fp8:
-        st.append(("quantize_rows", R * I * 2 + R * I + R * 8, 0))
+        st.append(("quantize_rows", R * I * 2 + R * I + R * 8, 0, 0))
     st += [
         ("grouped_down_gemm", down_w + H * S * 2 + R * I * wb + T * S * 2 + R * D * 2 + T * H * 4,
-         2 * R * I * D + 2 * T * S * H),
+         2 * R * I * D + 2 * T * S * H, f8 * 2 * R * I * D),
     ]
     if L:
-        st += [("latent_reduce", R * L * 2 + T * L * 2, 0),
-               ("fc2_gemm_blend", H * L * 2 + T * L * 2 + T * H * (4 + 2 + 2), 2 * T * L * H)]
+        st += [("latent_reduce", R * L * 2 + T * L * 2, 0, 0),
+               ("fc2_gemm_blend", H * L * 2 + T * L * 2 + T * H * (4 + 2 + 2), 2 * T * L * H, 0)]
     else:
-        st.append(("combine", R * D * 2 + T * H * 4 + T * H * 2 * 2, 0))
+        st.append(("combine", R * D * 2 + T * H * 4 + T * H * 2 * 2, 0, 0))
     return st
 
 
-def roofline_of(name, nbytes, flops, ms, peaks, expert_fp8):
+def step_work(s, T, U):
+    """What one forward must move and compute at least, whatever its kernels:
+    the gate, the U touched experts' weights, the shared expert, fc1/fc2, the
+    norm weight, and the token rows (hidden in, hidden out, residual out).
+    Returns (bytes, flops, fp8_flops)."""
+    H, E, k, I, S, L, D = s.H, s.E, s.k, s.I, s.S, s.L, s.D
+    R = T * k
+    wb = 1 if s.expert_fp8 else 2
+    scales = U * (I + D) * 4 if s.expert_fp8 else 0
+    nbytes = (E * H * 2 + U * 2 * D * I * wb + scales + 2 * H * S * 2 + 2 * H * L * 2 + H * 2
+              + 3 * T * H * 2)
+    routed = 4 * R * D * I
+    flops = 2 * T * H * E + routed + 4 * T * H * S + 4 * T * H * L
+    return nbytes, flops, (routed if s.expert_fp8 else 0)
+
+
+def roofline_of(name, nbytes, flops, ms, peaks, fp8_flops=0):
+    """The binding bound of `nbytes` and `flops` done in `ms`: HBM time at
+    the measured copy bandwidth, tensor time with the BF16 flops at the
+    measured BF16 peak and the FP8 flops at twice it (the nominal FP8/BF16
+    ratio), each class at its own rate.  frac = bound time / measured time."""
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    tf = peaks["bf16_tflops"] * (2.0 if expert_fp8 and "gemm" in name else 1.0)
-    t_tc = flops / (tf * 1e12) if flops else 0.0
+    bf = peaks["bf16_tflops"] * 1e12
+    t_tc = (flops - fp8_flops) / bf + fp8_flops / (2.0 * bf)
     if t_tc > t_hbm:
         ach = flops / (ms * 1e-3) / 1e12
-        return {"bound": "tensor", "achieved": round(ach, 2), "peak": tf, "unit": "TFLOP/s",
-                "frac": round(ach / tf, 4)}
+        peak = flops / t_tc / 1e12  # BF16 peak, 2x for FP8, mixed by flops
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(t_tc / (ms * 1e-3), 4)}
     ach = nbytes / (ms * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(ach / peaks["hbm_gbs"], 4)}
@@ -306,63 +333,58 @@ def config_of(s, T, path):
 
 # ------------------------------------------------------------------ ours ---
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
-    ap.add_argument("--tokens", type=int, default=None)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--eager", action="store_true",
-                    help="launch the forward eagerly each step instead of replaying a CUDA graph")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
+# Workloads measured after the headline one in the same run (N = 1), each at
+# the token count its configuration names; decode also at T = 8, the largest
+# batch of the decode path.
+SUB_WORKLOADS = (("decode", 8), ("tiny", 16), ("prefill", 1024), ("latent", 4096),
+                 ("skew_fp8", 8192))
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    shape = WORKLOADS[args.workload]
-    T = args.tokens or DEFAULT_TOKENS[args.workload]
+STAGE_NOTE = ("per-kernel times come from a second CUDA graph with events recorded between "
+              "the kernels; those events break the programmatic-dependent-launch overlap, so "
+              "the stage times sum to more than ms_per_step and each stage's frac is a lower bound")
 
-    if args.impl == "reference":
-        run_reference(args, shape, T, rank, world)
-        return
 
+class L2Flush:
+    """Writes 256 MB (evicting everything), then reads another 256 MB so L2
+    holds clean lines and the next step pays no write-backs."""
+
+    def __init__(self):
+        import torch
+        self.w = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+        self.r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+        self.out = torch.empty((), dtype=torch.float32, device="cuda")
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.amax(self.r, dim=0, out=self.out)
+
+
+def measure(inp, T, args, world, flush, peaks, *, e2e=True):
+    """Time `args.steps` forwards of T tokens of `inp` after `args.warmup`
+    untimed ones (CUDA-graph replay unless --eager, L2 flushed between
+    steps), on the device with CUDA events; the time is the max over ranks.
+    Returns the workload's record (throughput, roofline, stages, clocks,
+    end-to-end through the host-buffer entry point)."""
     import torch
     import torch.distributed as dist
 
     import mixture_experts_ffn_rmsnorm_b200 as moe
 
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    inp = make_inputs(shape, T=T)
+    shape = inp.shape
     layer = moe.MoELayer.from_inputs(inp, max_tokens=T)
-    path = "decode" if T <= 8 and shape.L == 0 and not shape.expert_fp8 else "prefill"
-    pristine = torch.from_numpy(inp.hidden.view(np.int16).copy()).cuda()
+    hbits = inp.hidden[:T]
+    pristine = torch.from_numpy(hbits.view(np.int16).copy()).cuda()
     hid = torch.empty_like(pristine)
     res = torch.empty_like(pristine)
-    flush_w = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-    flush_r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-    flush_out = torch.empty((), dtype=torch.float32, device="cuda")
-
-    def flush_l2():
-        # write 256 MB (evicts everything), then read another 256 MB so L2
-        # holds clean lines and the next step pays no write-backs
-        flush_w.zero_()
-        torch.amax(flush_r, dim=0, out=flush_out)
     stream = torch.cuda.current_stream()
 
-    # one untimed step to learn the launch count and the routing
+    # one untimed step to learn the launch count, the path and the routing
     hid.copy_(pristine)
     layer.forward(hid, res)
     torch.cuda.synchronize()
     nl = layer.last_launch_count()
+    path = "decode" if layer.last_path_decode() else "prefill"
     idx = torch.empty((T, shape.k), dtype=torch.int32, device="cuda")
     wts = torch.empty((T, shape.k), dtype=torch.float32, device="cuda")
     layer.copy_routing(idx, wts)
@@ -375,7 +397,7 @@ def main():
         return ev
 
     for _ in range(args.warmup):
-        flush_l2()
+        flush()
         hid.copy_(pristine)
         layer.forward(hid, res)
     torch.cuda.synchronize()
@@ -398,7 +420,7 @@ def main():
         layer.set_stage_events(None)
         stream.wait_stream(side)
         for _ in range(args.warmup):
-            flush_l2()
+            flush()
             hid.copy_(pristine)
             graph.replay()
         torch.cuda.synchronize()
@@ -409,9 +431,9 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(torch.cuda.current_device()) as clk:
         for i in range(args.steps):
-            flush_l2()
+            flush()
             hid.copy_(pristine)
             e_start[i].record(stream)
             if graph is not None:
@@ -426,6 +448,7 @@ def main():
     step_ms = np.array([a.elapsed_time(b) for a, b in zip(e_start, e_end)])
     total_ms = max_over_ranks(float(step_ms.sum()), world, "cuda")
     value = job_tokens_per_s(world, T, args.steps, total_ms)
+    ms_step = total_ms / args.steps
 
     # per-kernel device times: events recorded between the launches
     n_prof = min(args.steps, 50)
@@ -433,7 +456,7 @@ def main():
     if prof_graph is None:
         layer.set_stage_events(prof_events)
     for i in range(n_prof):
-        flush_l2()
+        flush()
         hid.copy_(pristine)
         if prof_graph is not None:
             prof_graph.replay()
@@ -443,31 +466,35 @@ def main():
         stage_ms[i] = [prof_events[j].elapsed_time(prof_events[j + 1]) for j in range(nl)]
     layer.set_stage_events(None)
 
-    # end to end through the host-buffer entry point (pinned host memory)
-    h_host = torch.from_numpy(inp.hidden.view(np.int16).copy()).pin_memory()
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    src = inp.hidden.view(np.int16)
-    for i in range(args.steps):
-        h_host.numpy()[...] = src
-        flush_l2()
-        e0[i].record(stream)
-        layer.forward_host(h_host)
-        e1[i].record(stream)
-        stream.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)), world, "cuda")
-    e2e = job_tokens_per_s(world, T, args.steps, e2e_ms)
+    e2e_rec = None
+    if e2e:
+        # end to end through the host-buffer entry point (pinned host memory)
+        h_host = torch.from_numpy(hbits.view(np.int16).copy()).pin_memory()
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        src = hbits.view(np.int16)
+        for i in range(args.steps):
+            h_host.numpy()[...] = src
+            flush()
+            e0[i].record(stream)
+            layer.forward_host(h_host)
+            e1[i].record(stream)
+            stream.synchronize()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)), world, "cuda")
+        e2e_rec = {"value": round(job_tokens_per_s(world, T, args.steps, e2e_ms), 2),
+                   "unit": UNIT, "h2d_bytes_per_step": T * shape.H * 2,
+                   "d2h_bytes_per_step": T * shape.H * 2}
+    layer.close()
 
-    peaks = measured_peaks()
     model = stage_model(shape, T, path, U)
     if path == "prefill" and len(model) + 1 == nl:
         model = stage_model(shape, T, path, U, router_split=True)
     if len(model) != nl:  # keep the JSON honest if the launch list changed
-        model = [(f"kernel_{j}", 0, 0) for j in range(nl)]
+        model = [(f"kernel_{j}", 0, 0, 0) for j in range(nl)]
     mean_stage = stage_ms.mean(axis=0)
     stages = []
-    for (name, nb, fl), ms in zip(model, mean_stage):
-        r = roofline_of(name, nb, fl, float(ms), peaks, shape.expert_fp8)
+    for (name, nb, fl, f8), ms in zip(model, mean_stage):
+        r = roofline_of(name, nb, fl, float(ms), peaks, f8)
         stages.append({"kernel": name, "ms": round(float(ms), 5),
                        "share": round(float(ms / mean_stage.sum()), 4), **r})
     dom = max(stages, key=lambda d: d["ms"])
@@ -476,30 +503,105 @@ def main():
     roof["kernel"] = dom["kernel"]
     roof["algorithmic"] = nb[1] if dom["bound"] == "hbm" else nb[2]
     roof["peak_source"] = peaks["source"] + (" (burst copy)" if dom["bound"] == "hbm"
-                                             else " bf16 burst")
+                                             else " bf16 burst, fp8 = 2x bf16")
     roof["traffic"] = kernel_traffic(dom["kernel"], f"{shape.name} T={T}")
+    wb, wf, w8 = step_work(shape, T, U)
+    step_roof = roofline_of("step", wb, wf, ms_step, peaks, w8)
+    step_roof.update({"algorithmic_bytes": wb, "algorithmic_flops": wf, "fp8_flops": w8,
+                      "note": "whole forward: gate, touched experts, shared expert, fc1/fc2 "
+                              "and token rows once, against ms_per_step"})
+    return {
+        "value": round(value, 2), "ms_per_step": round(ms_step, 5), "path": path,
+        "launch": "eager" if graph is None else "cuda_graph_replay", "distinct_experts": U,
+        "launches_per_step": nl, "clocks": clk.summary(), "e2e": e2e_rec, "roofline": roof,
+        "step_roofline": step_roof, "stages": stages, "stage_timing": STAGE_NOTE,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads' records (measured at N=1 only)")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the forward eagerly each step instead of replaying a CUDA graph")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    shape = WORKLOADS[args.workload]
+    T = args.tokens or DEFAULT_TOKENS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, shape, T, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    flush = L2Flush()
+    peaks = measured_peaks()
+    inp = make_inputs(shape, T=T)
+    rec = measure(inp, T, args, world, flush, peaks)
+
+    subs = []
+    if world == 1 and not args.no_workloads:
+        cache = {}
+        for name, Ts in SUB_WORKLOADS:
+            if name == args.workload and Ts == T:
+                continue
+            if name == args.workload and Ts <= T:
+                sub_inp = inp
+            else:
+                if name not in cache:
+                    cache.clear()
+                    cache[name] = make_inputs(WORKLOADS[name], T=Ts)
+                sub_inp = cache[name]
+            r = measure(sub_inp, Ts, args, world, flush, peaks)
+            subs.append({"workload": config_of(WORKLOADS[name], Ts, r["path"])["workload"],
+                         "tokens_per_step": Ts, "metric": METRIC, "unit": UNIT,
+                         "dtype": "fp8+bf16" if WORKLOADS[name].expert_fp8 else "bf16",
+                         "steps": args.steps, "warmup": args.warmup, **r})
+            del sub_inp
+        cache.clear()
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "metric": METRIC, "value": rec["value"], "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8+bf16" if shape.expert_fp8 else "bf16", "data": "synthetic",
-            "config": {**config_of(shape, T, path), "global_batch": world * T,
-                       "parallelism": f"replicas x{world}", "distinct_experts": U,
-                       "launch": "eager" if graph is None else "cuda_graph_replay"},
-            "clocks": clk.summary(),
-            "e2e": {"value": round(e2e, 2), "unit": UNIT,
-                    "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
-            "gpu_launches": nl * args.steps,
-            "roofline": roof,
-            "stages": stages,
+            "config": {**config_of(shape, T, rec["path"]), "global_batch": world * T,
+                       "parallelism": f"replicas x{world}",
+                       "distinct_experts": rec["distinct_experts"], "launch": rec["launch"]},
+            "clocks": rec["clocks"],
+            "e2e": rec["e2e"],
+            "gpu_launches": rec["launches_per_step"] * args.steps,
+            "roofline": rec["roofline"],
+            "step_roofline": rec["step_roofline"],
+            "stages": rec["stages"],
+            "stage_timing": STAGE_NOTE,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp, T)
+        if subs:
+            line["workloads"] = subs
         print(json.dumps(line), flush=True)
-    layer.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -87,18 +87,62 @@ def test_roofline_picks_the_binding_bound():
     peaks = {"hbm_gbs": 6530.0, "bf16_tflops": 1626.0, "bf16_tflops_sustained": 1399.0,
              "source": "measured"}
     # 80 MB in 30 us: HBM-bound, 2.67 TB/s
-    r = bench.roofline_of("decode_down_gemm", 80e6, 1e6, 0.030, peaks, False)
+    r = bench.roofline_of("decode_down_gemm", 80e6, 1e6, 0.030, peaks)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(80e6 / 30e-6 / 1e9, rel=1e-3)
     assert r["frac"] == pytest.approx(r["achieved"] / 6530.0, rel=1e-3)
-    # 800 GFLOP in 1 ms over 1.6 GB: tensor-bound; FP8 GEMMs get twice the peak
-    r = bench.roofline_of("grouped_up_gemm", 1.6e9, 800e9, 1.0, peaks, False)
+    # 800 GFLOP in 1 ms over 1.6 GB: tensor-bound
+    r = bench.roofline_of("grouped_up_gemm", 1.6e9, 800e9, 1.0, peaks)
     assert r["bound"] == "tensor" and r["peak"] == 1626.0
-    r8 = bench.roofline_of("grouped_up_gemm", 1.6e9, 800e9, 1.0, peaks, True)
+    assert r["frac"] == pytest.approx(800e9 / 1626e12 / 1e-3, rel=1e-3)
+    # all of it on FP8 operands: twice the peak, half the bound time
+    r8 = bench.roofline_of("grouped_up_gemm", 1.6e9, 800e9, 1.0, peaks, 800e9)
     assert r8["peak"] == 2 * 1626.0 and r8["frac"] == pytest.approx(r["frac"] / 2, rel=1e-3)
-    # non-GEMM kernels never take the FP8 factor
-    r = bench.roofline_of("combine", 1e8, 0, 0.02, peaks, True)
+    # kernels without flops are HBM-bound
+    r = bench.roofline_of("combine", 1e8, 0, 0.02, peaks)
     assert r["bound"] == "hbm"
+
+
+def test_mixed_fp8_bf16_launch_takes_each_class_at_its_own_peak():
+    # the skew workload's up launch at T = 8192: routed experts FP8, shared
+    # expert BF16 (same launch); the bound is the sum of the two classes'
+    # times, not all flops at the FP8 rate
+    peaks = {"hbm_gbs": 6530.0, "bf16_tflops": 1626.0, "source": "measured"}
+    s = WORKLOADS["skew_fp8"]
+    T = 8192
+    up = dict((m[0], m) for m in bench.stage_model(s, T, "prefill", s.E, router_split=True))[
+        "grouped_up_gemm"]
+    fp8 = 2 * T * s.k * s.H * s.I
+    bf16 = 2 * T * s.H * s.S
+    assert up[2] == fp8 + bf16 and up[3] == fp8
+    t_bound = fp8 / (2 * 1626e12) + bf16 / 1626e12
+    r = bench.roofline_of("grouped_up_gemm", up[1], up[2], 0.430, peaks, up[3])
+    assert r["bound"] == "tensor"
+    assert r["frac"] == pytest.approx(t_bound / 0.430e-3, rel=1e-3)
+    assert 0.55 < r["frac"] < 0.6   # 58 % at 430 us, where all-FP8 would say 47 %
+
+
+def test_gather_moves_each_token_row_once_and_writes_each_slot():
+    for name, T in (("prefill", 1024), ("skew_fp8", 8192), ("latent", 4096)):
+        s = WORKLOADS[name]
+        wb = 1 if s.expert_fp8 else 2
+        R = T * s.k
+        g = dict((m[0], m) for m in bench.stage_model(s, T, "prefill", s.E, True))["gather"]
+        assert g[1] == T * s.D * wb + R * s.D * wb + R * 4
+
+
+def test_step_work_closed_forms():
+    s = WORKLOADS["decode"]
+    nb, fl, f8 = bench.step_work(s, 1, 6)
+    assert nb == 160_355_328 and f8 == 0
+    assert fl == 2 * s.H * s.E + 4 * 6 * s.H * s.I + 4 * s.H * s.S
+    s = WORKLOADS["skew_fp8"]
+    nb, fl, f8 = bench.step_work(s, 8192, s.E)
+    assert f8 / 1e9 == pytest.approx(980.9, abs=0.05)
+    assert (fl - f8) / 1e9 == pytest.approx(332.6, abs=0.05)
+    s = WORKLOADS["latent"]
+    nb, fl, f8 = bench.step_work(s, 4096, s.E)
+    assert fl / 1e9 == pytest.approx(794.6, abs=0.05) and f8 == 0
 
 
 def test_committed_dram_captures_are_close_to_the_model():
