@@ -34,13 +34,15 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("I", ctypes.c_int32), ("S", ctypes.c_int32), ("L", ctypes.c_int32),
                 ("eps", ctypes.c_double), ("rsf", ctypes.c_double),
-                ("expert_fp8", ctypes.c_int32)]
+                ("expert_fp8", ctypes.c_int32), ("shared_fp8", ctypes.c_int32),
+                ("latent_fp8", ctypes.c_int32)]
 
 
 class _W(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("norm_w", "gate_w", "gate_bias", "up_w", "down_w", "up_scale",
-                 "down_scale", "shared_up_w", "shared_down_w", "fc1_w", "fc2_w")]
+                 "down_scale", "shared_up_w", "shared_down_w", "fc1_w", "fc2_w",
+                 "shared_up_scale", "shared_down_scale", "fc1_scale", "fc2_scale")]
 
 
 _lib = None
@@ -98,6 +100,8 @@ class Oracle:
             return a
 
         wd = np.uint8 if s.expert_fp8 else np.uint16
+        sd = np.uint8 if getattr(s, "shared_fp8", False) else np.uint16
+        ld = np.uint8 if getattr(s, "latent_fp8", False) else np.uint16
         arrs = dict(
             norm_w=c("norm_w", inp.norm_w, np.uint16),
             gate_w=c("gate_w", inp.gate_w, np.uint16),
@@ -106,13 +110,19 @@ class Oracle:
             down_w=c("down_w", inp.down_w, wd),
             up_scale=c("up_scale", inp.up_scale, np.float32),
             down_scale=c("down_scale", inp.down_scale, np.float32),
-            shared_up_w=c("shared_up_w", inp.shared_up_w, np.uint16),
-            shared_down_w=c("shared_down_w", inp.shared_down_w, np.uint16),
-            fc1_w=c("fc1_w", inp.fc1_w, np.uint16),
-            fc2_w=c("fc2_w", inp.fc2_w, np.uint16),
+            shared_up_w=c("shared_up_w", inp.shared_up_w, sd),
+            shared_down_w=c("shared_down_w", inp.shared_down_w, sd),
+            fc1_w=c("fc1_w", inp.fc1_w, ld),
+            fc2_w=c("fc2_w", inp.fc2_w, ld),
+            shared_up_scale=c("shared_up_scale", getattr(inp, "shared_up_scale", None), np.float32),
+            shared_down_scale=c("shared_down_scale", getattr(inp, "shared_down_scale", None),
+                                np.float32),
+            fc1_scale=c("fc1_scale", getattr(inp, "fc1_scale", None), np.float32),
+            fc2_scale=c("fc2_scale", getattr(inp, "fc2_scale", None), np.float32),
         )
         self.cfg = _Cfg(s.H, s.E, s.k, s.I, s.S, s.L, float(s.eps), float(s.rsf),
-                        1 if s.expert_fp8 else 0)
+                        1 if s.expert_fp8 else 0, 1 if sd is np.uint8 else 0,
+                        1 if ld is np.uint8 else 0)
         self.w = _W(**{k: (None if v is None else v.ctypes.data) for k, v in arrs.items()})
         self.bias = arrs["gate_bias"]
 

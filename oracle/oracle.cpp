@@ -31,7 +31,11 @@
 //   R7 the shared expert is unweighted and works on the normed vector in H;
 //   R8 LatentMoE: gate on the normed vector, fc1 on the normed vector, the
 //      weighted sum in latent space, then fc2;
-//   R9 the norm weight multiplies directly (x * r * w).
+//   R9 the norm weight multiplies directly (x * r * w);
+//   R10 FP8 weights (routed experts, and optionally the shared expert and
+//      fc1 / fc2, which the pages also keep as FP8 copies: nemotron_moe.rs
+//      `new`) are E4M3 bytes times one float32 scale per output row, taken
+//      exactly; activations are never quantised here.
 // Parity pins: tests/test_oracle_pins.py (closed forms, brute-force subset
 // enumeration, hand-computed cases, invariants).
 #include <cmath>
@@ -48,6 +52,8 @@ typedef struct {
   double eps;                // rms_norm_eps
   double rsf;                // routed_scaling_factor
   int32_t expert_fp8;        // 0: routed weights BF16; 1: FP8 E4M3 + FP32 row scale
+  int32_t shared_fp8;        // shared expert weights: 0 BF16, 1 FP8 E4M3 + FP32 row scale
+  int32_t latent_fp8;        // fc1 / fc2 weights: 0 BF16, 1 FP8 E4M3 + FP32 row scale
 } oracle_cfg;
 
 typedef struct {
@@ -58,10 +64,14 @@ typedef struct {
   const void* down_w;             // [E,D,I] bf16 or e4m3
   const float* up_scale;          // [E,I]  (fp8 only)
   const float* down_scale;        // [E,D]  (fp8 only)
-  const uint16_t* shared_up_w;    // [S,H]  bf16
-  const uint16_t* shared_down_w;  // [H,S]  bf16
-  const uint16_t* fc1_w;          // [L,H]  bf16 (latent only)
-  const uint16_t* fc2_w;          // [H,L]  bf16 (latent only)
+  const void* shared_up_w;        // [S,H]  bf16 or e4m3
+  const void* shared_down_w;      // [H,S]  bf16 or e4m3
+  const void* fc1_w;              // [L,H]  bf16 or e4m3 (latent only)
+  const void* fc2_w;              // [H,L]  bf16 or e4m3 (latent only)
+  const float* shared_up_scale;   // [S]    (shared_fp8 only)
+  const float* shared_down_scale; // [H]    (shared_fp8 only)
+  const float* fc1_scale;         // [L]    (latent_fp8 only)
+  const float* fc2_scale;         // [H]    (latent_fp8 only)
 } oracle_weights;
 
 }  // extern "C"
@@ -107,6 +117,15 @@ double expert_w(const oracle_cfg& c, const void* w, const float* scale,
   size_t i = (size_t(e) * rows + r) * size_t(cols) + col;
   if (c.expert_fp8)
     return kE4M3.v[static_cast<const uint8_t*>(w)[i]] * double(scale[size_t(e) * rows + r]);
+  return bf16(static_cast<const uint16_t*>(w)[i]);
+}
+
+// Element (r, col) of a dense [rows, cols] weight (shared expert, fc1,
+// fc2), dequantised the same way as the routed experts when fp8 is set:
+// e4m3 value times the row's scale.
+double dense_w(const void* w, const float* scale, int fp8, int r, int col, int cols) {
+  size_t i = size_t(r) * size_t(cols) + col;
+  if (fp8) return kE4M3.v[static_cast<const uint8_t*>(w)[i]] * double(scale[r]);
   return bf16(static_cast<const uint16_t*>(w)[i]);
 }
 
@@ -184,7 +203,7 @@ void token_forward(const oracle_cfg& c, const oracle_weights& w, const uint16_t*
   if (c.L > 0) {
     for (int l = 0; l < c.L; ++l) {
       double a = 0.0;
-      for (int i = 0; i < H; ++i) a += n[i] * bf16(w.fc1_w[size_t(l) * H + i]);
+      for (int i = 0; i < H; ++i) a += n[i] * dense_w(w.fc1_w, w.fc1_scale, c.latent_fp8, l, i, H);
       z[l] = a;
     }
   } else {
@@ -198,7 +217,7 @@ void token_forward(const oracle_cfg& c, const oracle_weights& w, const uint16_t*
   if (c.L > 0) {
     for (int h = 0; h < H; ++h) {
       double a = 0.0;
-      for (int l = 0; l < c.L; ++l) a += m[l] * bf16(w.fc2_w[size_t(h) * c.L + l]);
+      for (int l = 0; l < c.L; ++l) a += m[l] * dense_w(w.fc2_w, w.fc2_scale, c.latent_fp8, h, l, c.L);
       routed[h] = a;
     }
   } else {
@@ -206,12 +225,12 @@ void token_forward(const oracle_cfg& c, const oracle_weights& w, const uint16_t*
   }
   for (int s = 0; s < c.S; ++s) {
     double a = 0.0;
-    for (int i = 0; i < H; ++i) a += n[i] * bf16(w.shared_up_w[size_t(s) * H + i]);
+    for (int i = 0; i < H; ++i) a += n[i] * dense_w(w.shared_up_w, w.shared_up_scale, c.shared_fp8, s, i, H);
     v[s] = relu2(a);
   }
   for (int h = 0; h < H; ++h) {
     double a = 0.0;
-    for (int s = 0; s < c.S; ++s) a += v[s] * bf16(w.shared_down_w[size_t(h) * c.S + s]);
+    for (int s = 0; s < c.S; ++s) a += v[s] * dense_w(w.shared_down_w, w.shared_down_scale, c.shared_fp8, h, s, c.S);
     out[h] = bf16(x[h]) + routed[h] + a;
   }
 }
@@ -325,6 +344,8 @@ int oracle_forward(const oracle_cfg* c, const oracle_weights* w, const uint16_t*
   if (check_cfg(c) || T < 0) return 1;
   if (c->L > 0 && (!w->fc1_w || !w->fc2_w)) return 1;
   if (c->expert_fp8 && (!w->up_scale || !w->down_scale)) return 1;
+  if (c->shared_fp8 && (!w->shared_up_scale || !w->shared_down_scale)) return 1;
+  if (c->L > 0 && c->latent_fp8 && (!w->fc1_scale || !w->fc2_scale)) return 1;
   parallel_tokens(T, nthreads, [&](int t) {
     token_forward(*c, *w, hidden + size_t(t) * c->H,
                   forced_idx ? forced_idx + size_t(t) * c->k : nullptr,

@@ -35,7 +35,10 @@ def numpy_layer(inp, hidden_bits):
             return e4m3_to_f32(m).astype(np.float64) * scale[:, None]
         return _f64_bf16(m)
 
-    z = n if not s.L else n @ _f64_bf16(inp.fc1_w).T
+    def dense(m, scale, fp8):  # shared expert / fc1 / fc2 weights as float64 [out, in]
+        return e4m3_to_f32(m).astype(np.float64) * scale[:, None] if fp8 else _f64_bf16(m)
+
+    z = n if not s.L else n @ dense(inp.fc1_w, inp.fc1_scale, s.latent_fp8).T
     m = np.zeros_like(z)
     for t in range(T):
         for j in range(k):
@@ -45,9 +48,9 @@ def numpy_layer(inp, hidden_bits):
             u = np.maximum(up @ z[t], 0.0) ** 2
             m[t] += w[t, j] * (dn @ u)
     if s.L:
-        m = m @ _f64_bf16(inp.fc2_w).T
-    v = np.maximum(n @ _f64_bf16(inp.shared_up_w).T, 0.0) ** 2
-    return x + m + v @ _f64_bf16(inp.shared_down_w).T, idx, w
+        m = m @ dense(inp.fc2_w, inp.fc2_scale, s.latent_fp8).T
+    v = np.maximum(n @ dense(inp.shared_up_w, inp.shared_up_scale, s.shared_fp8).T, 0.0) ** 2
+    return x + m + v @ dense(inp.shared_down_w, inp.shared_down_scale, s.shared_fp8).T, idx, w
 
 
 @pytest.mark.parametrize("name,T,over", [
@@ -55,6 +58,8 @@ def numpy_layer(inp, hidden_bits):
     ("decode", 8, {}),
     ("latent", 6, dict(H=512, I=256, S=512, L=256)),
     ("skew_fp8", 8, dict(H=512, I=256, S=512, E=32)),
+    ("skew_fp8", 8, dict(H=512, I=256, S=512, E=32, shared_fp8=True)),
+    ("latent", 6, dict(H=512, I=256, S=512, L=256, shared_fp8=True, latent_fp8=True)),
 ])
 def test_oracle_matches_numpy_restatement(name, T, over):
     shape = WORKLOADS[name].scaled(**over) if over else WORKLOADS[name]

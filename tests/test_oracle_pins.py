@@ -398,3 +398,38 @@ def test_route_weights_of_forced_sets_match_the_scores():
     # the oracle's own choice gives its own weights
     idx, ow, _ = o.route(lg)
     np.testing.assert_array_equal(o.route_weights(lg, idx), ow)
+
+
+@pytest.mark.parametrize("which", ["shared", "latent"])
+def test_fp8_dense_weights_equal_bf16_when_dequantised_values_are_exact(which):
+    # Shared expert (up, down) or LatentMoE fc1 / fc2 stored as E4M3 codes
+    # with power-of-two row scales: the dequantised values are exact in
+    # BF16, so the FP8 oracle must reproduce the BF16 oracle run on them.
+    # A missing row scale or a transposed scale index changes the result.
+    from workloads import e4m3_to_f32
+    base = WORKLOADS["tiny"].scaled(T=6, L=64 if which == "latent" else 0)
+    d = make_inputs(base)
+    rng = np.random.default_rng(11)
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    names = ("shared_up", "shared_down") if which == "shared" else ("fc1", "fc2")
+    f8 = make_inputs(base.scaled(**{f"{which}_fp8": True}))
+    for name in ("norm_w", "gate_w", "gate_bias", "up_w", "down_w", "hidden",
+                 "shared_up_w", "shared_down_w", "fc1_w", "fc2_w"):
+        setattr(f8, name, getattr(d, name))
+    for n in names:
+        w = getattr(d, f"{n}_w")
+        qc = rng.choice(codes, size=w.shape).astype(np.uint8)
+        sc = (2.0 ** -rng.integers(3, 8, size=w.shape[0])).astype(np.float32)
+        setattr(f8, f"{n}_w", qc)
+        setattr(f8, f"{n}_scale", sc)
+        setattr(d, f"{n}_w", exact_bf16(e4m3_to_f32(qc).astype(np.float64) * sc[:, None]))
+    o8, i8, _ = oracle.Oracle(f8).forward(f8.hidden)
+    ob, ib, _ = oracle.Oracle(d).forward(d.hidden)
+    np.testing.assert_array_equal(i8, ib)
+    np.testing.assert_array_equal(o8, ob)
+    # and the FP8 weights do matter: a changed row scale changes the output
+    sc = getattr(f8, f"{names[1]}_scale").copy()
+    sc[0] *= 2.0
+    setattr(f8, f"{names[1]}_scale", sc)
+    o8b, _, _ = oracle.Oracle(f8).forward(f8.hidden)
+    assert not np.array_equal(o8b, o8)

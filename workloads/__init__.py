@@ -46,6 +46,8 @@ class MoEShape:
     rsf: float = 1.0  # routed_scaling_factor
     eps: float = 1e-5
     expert_fp8: bool = False   # routed up/down stored as FP8 E4M3 + FP32 row scale
+    shared_fp8: bool = False   # shared expert up/down stored the same way
+    latent_fp8: bool = False   # fc1 / fc2 stored the same way
     bias: str = "none"         # "none" | "uniform" (U(-0.1,0.1)) | "zipf"
     gate_scale: float = 1.0    # gate ~ N(0, gate_scale / H)
     seed: int = 0
@@ -180,6 +182,10 @@ class Inputs:
     fc2_w: Optional[np.ndarray]          # [H,L] bf16 bits
     hidden: np.ndarray                   # [T,H] bf16 bits
     residual: np.ndarray                 # [T,H] bf16 bits (ignored by the layer)
+    shared_up_scale: Optional[np.ndarray] = None    # [S] float32 (shared_fp8 only)
+    shared_down_scale: Optional[np.ndarray] = None  # [H] float32 (shared_fp8 only)
+    fc1_scale: Optional[np.ndarray] = None          # [L] float32 (latent_fp8 only)
+    fc2_scale: Optional[np.ndarray] = None          # [H] float32 (latent_fp8 only)
 
 
 def _normal(rng, shape, std):
@@ -251,16 +257,20 @@ def make_inputs(shape: MoEShape, T: Optional[int] = None,
     D = s.D
     up_w = down_w = up_scale = down_scale = None
     shared_up_w = shared_down_w = fc1_w = fc2_w = None
+    shared_up_scale = shared_down_scale = fc1_scale = fc2_scale = None
     if experts:
         up_w, up_scale = _expert_stack(seqs["up"], s.E, s.I, D, s.expert_fp8)
         down_w, down_scale = _expert_stack(seqs["down"], s.E, D, s.I, s.expert_fp8)
-        shared_up_w = bf16_bits(_normal(rng["shared_up"], (s.S, s.H), 1.0 / np.sqrt(s.H)))
-        shared_down_w = bf16_bits(_normal(rng["shared_down"], (s.H, s.S), 1.0 / np.sqrt(s.S)))
+        def dense(name, rows, cols, fp8):
+            x = _normal(rng[name], (rows, cols), 1.0 / np.sqrt(cols))
+            return _quantize_rows_e4m3(x) if fp8 else (bf16_bits(x), None)
+        shared_up_w, shared_up_scale = dense("shared_up", s.S, s.H, s.shared_fp8)
+        shared_down_w, shared_down_scale = dense("shared_down", s.H, s.S, s.shared_fp8)
         if s.L > 0:
-            fc1_w = bf16_bits(_normal(rng["fc1"], (s.L, s.H), 1.0 / np.sqrt(s.H)))
-            fc2_w = bf16_bits(_normal(rng["fc2"], (s.H, s.L), 1.0 / np.sqrt(s.L)))
+            fc1_w, fc1_scale = dense("fc1", s.L, s.H, s.latent_fp8)
+            fc2_w, fc2_scale = dense("fc2", s.H, s.L, s.latent_fp8)
     hidden = bf16_bits(_normal(rng["hidden"], (s.T, s.H), 1.0))
     residual = bf16_bits(_normal(rng["residual"], (s.T, s.H), 1.0))
     return Inputs(s, norm_w, gate_w, gate_bias, up_w, down_w, up_scale,
                   down_scale, shared_up_w, shared_down_w, fc1_w, fc2_w,
-                  hidden, residual)
+                  hidden, residual, shared_up_scale, shared_down_scale, fc1_scale, fc2_scale)
