@@ -78,13 +78,10 @@ def stage_model(s, T, path, U, router_split=False):
     down_w = U * D * I * wb + (U * D * 4 if s.expert_fp8 else 0)
     f8 = 1 if s.expert_fp8 else 0
     if path == "decode":
-        return [
-            ("decode_route", E * H * 2 + 3 * T * H * 2 + T * E * 4, 2 * T * H * E, 0),
-            ("decode_up_gemm", up_w + S * H * 2 + T * H * 2 + R * I * 2 + T * S * 2,
-             2 * R * D * I + 2 * T * H * S, f8 * 2 * R * D * I),
-            ("decode_down_gemm", down_w + H * S * 2 + R * I * 2 + T * S * 2 + T * H * 2 * 2,
-             2 * R * I * D + 2 * T * S * H, f8 * 2 * R * I * D),
-        ]
+        # one launch: the whole forward (its up outputs and partial sums stay
+        # in L2 and are not counted)
+        nb, fl, f8f = step_work(s, T, U)
+        return [("decode_fused", nb, fl, f8f)]
     st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2 + (T * H if s.expert_fp8 else 0), 0, 0)]
     # With split K (few token tiles) the router GEMM stores partial logits
     # and a second kernel sums them and selects; its algorithmic bytes are

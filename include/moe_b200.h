@@ -67,8 +67,8 @@ typedef enum {
 } moe_status;
 
 typedef enum {
-  MOE_WEIGHTS_BF16 = 0,            /* routed up/down stored as BF16 */
-  MOE_WEIGHTS_FP8_E4M3_ROWSCALE = 1/* routed up/down as E4M3 + float32 scale per output row */
+  MOE_WEIGHTS_BF16 = 0,            /* stored as BF16 */
+  MOE_WEIGHTS_FP8_E4M3_ROWSCALE = 1/* stored as E4M3 + float32 scale per output row */
 } moe_weight_dtype;
 
 /* Routing-kernel bounds (NemotronMoeLayer `new` refuses a top_k outside
@@ -86,7 +86,11 @@ typedef enum {
  *   num_experts <= MOE_MAX_EXPERTS, max_tokens >= 1,
  *   hidden_size, moe_inter, shared_inter, latent_size all multiples of 64
  *   (latent_size may be 0), rms_eps >= 0, routed_scaling_factor finite,
- *   expert_wdtype a moe_weight_dtype value. */
+ *   expert_wdtype, shared_wdtype and latent_wdtype moe_weight_dtype values,
+ *   and not FP8 routed experts together with latent_size > 0.
+ * FP8 weights (nemotron_moe.rs `new` keeps FP8 copies of the routed
+ * experts, the shared expert and fc1 / fc2) run as W8A8 on the tensor
+ * cores: their input rows are quantised to E4M3 with one scale per row. */
 typedef struct {
   int32_t hidden_size;           /* H */
   int32_t num_experts;           /* E */
@@ -97,7 +101,9 @@ typedef struct {
   int32_t max_tokens;            /* largest num_tokens a forward call may pass */
   float rms_eps;                 /* RMSNorm epsilon */
   float routed_scaling_factor;   /* multiplies the renormalised routing weights */
-  int32_t expert_wdtype;         /* moe_weight_dtype */
+  int32_t expert_wdtype;         /* moe_weight_dtype of the routed experts' up / down */
+  int32_t shared_wdtype;         /* moe_weight_dtype of the shared expert's up / down */
+  int32_t latent_wdtype;         /* moe_weight_dtype of fc1 / fc2 (latent layers) */
 } moe_config;
 
 /* Device pointers to the layer's weights (all borrowed, 16-byte aligned). */
@@ -109,10 +115,14 @@ typedef struct {
   const void* down_w;        /* [E, D, I] bf16 or e4m3 */
   const float* up_scale;     /* [E, I] f32, FP8 only (else NULL) */
   const float* down_scale;   /* [E, D] f32, FP8 only (else NULL) */
-  const void* shared_up_w;   /* [S, H] bf16 */
-  const void* shared_down_w; /* [H, S] bf16 */
-  const void* fc1_w;         /* [L, H] bf16, latent only (else NULL) */
-  const void* fc2_w;         /* [H, L] bf16, latent only (else NULL) */
+  const void* shared_up_w;   /* [S, H] bf16 or e4m3 */
+  const void* shared_down_w; /* [H, S] bf16 or e4m3 */
+  const void* fc1_w;         /* [L, H] bf16 or e4m3, latent only (else NULL) */
+  const void* fc2_w;         /* [H, L] bf16 or e4m3, latent only (else NULL) */
+  const float* shared_up_scale;   /* [S] f32, FP8 shared expert only (else NULL) */
+  const float* shared_down_scale; /* [H] f32, FP8 shared expert only (else NULL) */
+  const float* fc1_scale;         /* [L] f32, FP8 fc1 / fc2 only (else NULL) */
+  const float* fc2_scale;         /* [H] f32, FP8 fc1 / fc2 only (else NULL) */
 } moe_weights;
 
 typedef struct moe_handle moe_handle;
@@ -243,7 +253,9 @@ MOE_API moe_status moe_copy_sort(moe_handle* h, int32_t* perm, int32_t* inv, int
                                  int32_t num_tokens, void* stream);
 
 /* Copy the device status word into *status (0 = no device-side timeout) and
- * clear it.  Synchronises the stream (debug use only). */
+ * clear it; after a non-zero status also reset the handle's device-side
+ * tile and schedule counters, which a pass that gave up may have left
+ * mid-count.  Synchronises the stream (debug use only). */
 MOE_API moe_status moe_get_device_status(moe_handle* h, int32_t* status, void* stream);
 
 /* Profiling: every following moe_forward* call records caller-owned CUDA

@@ -42,13 +42,15 @@ class MoEConfig(ctypes.Structure):
                 ("top_k", ctypes.c_int32), ("moe_inter", ctypes.c_int32),
                 ("shared_inter", ctypes.c_int32), ("latent_size", ctypes.c_int32),
                 ("max_tokens", ctypes.c_int32), ("rms_eps", ctypes.c_float),
-                ("routed_scaling_factor", ctypes.c_float), ("expert_wdtype", ctypes.c_int32)]
+                ("routed_scaling_factor", ctypes.c_float), ("expert_wdtype", ctypes.c_int32),
+                ("shared_wdtype", ctypes.c_int32), ("latent_wdtype", ctypes.c_int32)]
 
 
 class MoEWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("norm_w", "gate_w", "gate_bias", "up_w", "down_w", "up_scale", "down_scale",
-                 "shared_up_w", "shared_down_w", "fc1_w", "fc2_w")]
+                 "shared_up_w", "shared_down_w", "fc1_w", "fc2_w", "shared_up_scale",
+                 "shared_down_scale", "fc1_scale", "fc2_scale")]
 
 
 _lib = None
@@ -127,16 +129,21 @@ class MoELayer:
 
     def __init__(self, *, hidden_size, num_experts, top_k, moe_inter, shared_inter,
                  latent_size=0, max_tokens, rms_eps=1e-5, routed_scaling_factor=1.0,
-                 expert_fp8=False, norm_w, gate_w, gate_bias=None, up_w, down_w, up_scale=None,
-                 down_scale=None, shared_up_w, shared_down_w, fc1_w=None, fc2_w=None):
+                 expert_fp8=False, shared_fp8=False, latent_fp8=False, norm_w, gate_w,
+                 gate_bias=None, up_w, down_w, up_scale=None, down_scale=None, shared_up_w,
+                 shared_down_w, fc1_w=None, fc2_w=None, shared_up_scale=None,
+                 shared_down_scale=None, fc1_scale=None, fc2_scale=None):
         self.lib = load_library()
+        dt = lambda f: WEIGHTS_FP8 if f else WEIGHTS_BF16  # noqa: E731
         self.cfg = MoEConfig(hidden_size, num_experts, top_k, moe_inter, shared_inter,
                              latent_size, max_tokens, rms_eps, routed_scaling_factor,
-                             WEIGHTS_FP8 if expert_fp8 else WEIGHTS_BF16)
+                             dt(expert_fp8), dt(shared_fp8), dt(latent_fp8))
         self._tensors = dict(norm_w=norm_w, gate_w=gate_w, gate_bias=gate_bias, up_w=up_w,
                              down_w=down_w, up_scale=up_scale, down_scale=down_scale,
                              shared_up_w=shared_up_w, shared_down_w=shared_down_w,
-                             fc1_w=fc1_w, fc2_w=fc2_w)
+                             fc1_w=fc1_w, fc2_w=fc2_w, shared_up_scale=shared_up_scale,
+                             shared_down_scale=shared_down_scale, fc1_scale=fc1_scale,
+                             fc2_scale=fc2_scale)
         self.w = MoEWeights(**{k: _ptr(v) for k, v in self._tensors.items()})
         self.handle = ctypes.c_void_p()
         st = self.lib.moe_create(ctypes.byref(self.cfg), ctypes.byref(self.w),
@@ -232,13 +239,22 @@ class MoELayer:
 
         s = inp.shape
         b16 = np.int16
+        sf8, lf8 = getattr(s, "shared_fp8", False), getattr(s, "latent_fp8", False)
         wd = np.uint8 if s.expert_fp8 else b16
+        sd = np.uint8 if sf8 else b16
+        ld = np.uint8 if lf8 else b16
+        f32 = np.float32
         return cls(hidden_size=s.H, num_experts=s.E, top_k=s.k, moe_inter=s.I,
                    shared_inter=s.S, latent_size=s.L, max_tokens=max_tokens or s.T,
                    rms_eps=s.eps, routed_scaling_factor=s.rsf, expert_fp8=s.expert_fp8,
+                   shared_fp8=sf8, latent_fp8=lf8,
                    norm_w=up(inp.norm_w, b16), gate_w=up(inp.gate_w, b16),
-                   gate_bias=up(inp.gate_bias, np.float32), up_w=up(inp.up_w, wd),
-                   down_w=up(inp.down_w, wd), up_scale=up(inp.up_scale, np.float32),
-                   down_scale=up(inp.down_scale, np.float32),
-                   shared_up_w=up(inp.shared_up_w, b16), shared_down_w=up(inp.shared_down_w, b16),
-                   fc1_w=up(inp.fc1_w, b16), fc2_w=up(inp.fc2_w, b16))
+                   gate_bias=up(inp.gate_bias, f32), up_w=up(inp.up_w, wd),
+                   down_w=up(inp.down_w, wd), up_scale=up(inp.up_scale, f32),
+                   down_scale=up(inp.down_scale, f32),
+                   shared_up_w=up(inp.shared_up_w, sd), shared_down_w=up(inp.shared_down_w, sd),
+                   fc1_w=up(inp.fc1_w, ld), fc2_w=up(inp.fc2_w, ld),
+                   shared_up_scale=up(getattr(inp, "shared_up_scale", None), f32),
+                   shared_down_scale=up(getattr(inp, "shared_down_scale", None), f32),
+                   fc1_scale=up(getattr(inp, "fc1_scale", None), f32),
+                   fc2_scale=up(getattr(inp, "fc2_scale", None), f32))

@@ -1,0 +1,1042 @@
+// Decode path (1 <= T <= 8 tokens) as ONE persistent launch.
+//
+// At these sizes the layer streams weights (NemotronMoeLayer `decode`;
+// MoeLayer `forward_k2` / `forward_k3` run a few tokens through one weight
+// sweep): about 160 MB at T = 1 against a few MFLOP.  The pass runs as one
+// cooperative grid of one CTA per SM.
+//
+// The work is cut along the experts' intermediate dimension.  A unit is 128
+// intermediate rows of one expert (the shared expert's, or a routed slot's):
+//   up     u = relu^2(W_up[rows] . n) (x routing weight), 128 x 16 tokens,
+//          K = H: tcgen05.mma M = 128 (weight rows), N = 16 (tokens), BF16 in,
+//          fp32 accumulate in TMEM;
+//   down   y += W_down[:, rows] . u over all H output rows (K = 128), the
+//          relu^2 rows going from TMEM through shared memory as the MMA's
+//          token operand.
+// A unit needs nothing from other CTAs once the tokens are routed, and every
+// unit's down adds into the same H x 16 accumulator, which stays in TMEM
+// (ceil(H / 128) x 16 columns) until the CTA's last unit.  Unit j goes to
+// CTA j % grid: shared-expert units first (they need no routing and start at
+// once), routed units after.  At the end every CTA stores its partial H x T
+// block, and each CTA adds up one slice of rows over all CTAs' partials, in
+// CTA order (deterministic), plus the residual, into hidden.
+//
+// Warp roles (320 threads):
+//   warp 0     TMA producer: weight boxes (and the up GEMM's token rows) into
+//              a ring of stages; up and down boxes interleave so a unit's
+//              relu^2 rows are ready by the time its down boxes are consumed.
+//   warp 1     TMEM owner and MMA issuer.
+//   warps 2-5  epilogue: relu^2 rows into shared memory; the partial output.
+//   warps 6-9  routing: one pass over this CTA's gate row(s) and the tokens
+//              gives the sums of squares and the dot products at once,
+//              logit = rsqrt(mean x^2 + eps) * (G_e . (x * w)) in fp32, and
+//              the CTA's own copy of the bf16 normed rows (the up GEMM's token
+//              operand); CTA 0 writes the residual.  Once every CTA's logits
+//              are in, each CTA runs the same sigmoid top-k and builds the
+//              same table of routed slots (distinct experts, first-use order).
+//   all        the final reduction.
+//
+// Every wait is bounded (about one second): a timeout sets a status bit, the
+// CTA drains its own TMA loads and MMAs, frees its TMEM and returns.
+#include "decode.h"
+#include "ptx.cuh"
+#include "topk.cuh"
+
+namespace moe {
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kStages = 11;
+constexpr int kABytes = kBM * 128;          // 128 weight rows x 64 BF16
+constexpr int kBBytes = kDecodeN * 128;     // 16 token rows x 64 BF16
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kUBytes = 2 * kBBytes;        // a unit's relu^2 rows: 16 tokens x 128 K, two 64-wide chunks
+constexpr int kThreads = 320;               // see the warp roles above
+constexpr int kEpiThreads = 128;
+constexpr int kRouteThreads = 128;
+constexpr int kMaxSlots = kDecodeMaxT * kTopKMax;  // routed slots (distinct experts)
+constexpr int kMaxChunks = 4;               // 8-element chunks per routing thread (H <= 4096)
+constexpr int kTmemCols = 512;              // 2 x 16 (up) + ceil(H / 128) x 16 (down)
+constexpr int kMaxRowTiles = kTmemCols / kDecodeN - 2;
+constexpr int kSmem = kStages * kStageBytes + 2 * kUBytes + 1024 + 1024;
+
+// Named barriers (0 is __syncthreads).
+constexpr int kBarEpi = 1;
+constexpr int kBarRoute = 2;
+
+// Synchronisation words of the workspace (FusedWorkspace::sync).
+enum { kRouteArrived = 0, kPartialsDone = 1, kExited = 2 };
+
+struct FusedParams {
+  CUtensorMap tm_up;     // routed up weights   [E*I, H]  (A, 128-row boxes)
+  CUtensorMap tm_sup;    // shared up weights   [S, H]
+  CUtensorMap tm_down;   // routed down weights [E*H, I]
+  CUtensorMap tm_sdown;  // shared down weights [H, S]
+  CUtensorMap tm_x;      // x16 [grid * 16, H]: 16 rows per CTA   (B, 16-row boxes)
+  const bf16* hidden;
+  bf16* residual;
+  bf16* out;             // = hidden (written at the very end)
+  const bf16* norm_w;
+  const bf16* gate_w;
+  const float* gate_bias;
+  int T, H, E, k, I, S;
+  float eps, rsf;
+  FusedWorkspace ws;
+  int* status;
+};
+
+// ------------------------------------------------- memory-model helpers
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Release increment: this thread's earlier writes, and those of the threads
+// it synchronised with through a barrier, become visible before the count.
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Order this thread's generic-proxy global accesses with its later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Make this thread's shared-memory writes visible to the tensor cores.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void record_timeout(int* status, volatile int* abort) {
+  *abort = 1;
+  if (status) atomicOr(status, kStatusWaitTimeout);
+}
+
+// Bounded wait until *p >= target (acquire), polling every ~100 ns.  False
+// on timeout or abort.
+__device__ __forceinline__ bool wait_counter(const unsigned* p, unsigned target,
+                                             volatile int* abort) {
+  if (ld_acquire(p) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(100);
+    if (ld_acquire(p) >= target) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+  }
+}
+
+__device__ __forceinline__ float lo16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  f[0] = lo16(u.x); f[1] = hi16(u.x);
+  f[2] = lo16(u.y); f[3] = hi16(u.y);
+  f[4] = lo16(u.z); f[5] = hi16(u.z);
+  f[6] = lo16(u.w); f[7] = hi16(u.w);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Shared state of one CTA.
+struct Shared {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t tfull[2], tempty[2];   // up accumulators: MMA -> epilogue -> MMA
+  uint64_t ufull[2], ufree[2];    // relu^2 row buffers: epilogue -> MMA -> epilogue
+  uint64_t down_done;             // every down MMA of the CTA has completed
+  uint64_t loads_out;             // the routing warps' loads have returned
+  uint64_t tokens;                // this CTA's normed rows are written (TMA may load them)
+  uint64_t routed;                // the routing warps have built the slot table
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int stop;                 // the epilogue warps' common decision to stop (epi_stop)
+  int route_fail;
+  int flag;
+  int U;                    // routed slots
+  float rs[kDecodeMaxT];
+  float red[4][kDecodeMaxT * 3];
+  int seg_expert[kMaxSlots];            // expert of routed slot s
+  float seg_w[kMaxSlots][kDecodeN];     // routing weight of token t in slot s (0 = not routed)
+  int sel_idx[kDecodeMaxT * kTopKMax];
+  float sel_w[kDecodeMaxT * kTopKMax];
+  int first_use[kDecodeMaxT * kTopKMax];
+  int slot_of[MOE_MAX_EXPERTS];
+  float bias[MOE_MAX_EXPERTS];
+};
+
+static_assert(kSmem + sizeof(Shared) <= 227 * 1024, "shared memory of one CTA");
+
+// The four epilogue warps meet here and take one decision together:
+// whether to stop (some role recorded a timeout).  Control flow of the
+// epilogue warps never diverges, so their named barriers always complete.
+__device__ __forceinline__ bool epi_stop(Shared& sh, int tid) {
+  named_barrier(kBarEpi, kEpiThreads);
+  if (tid == 0) sh.stop = sh.abort;
+  named_barrier(kBarEpi, kEpiThreads);
+  return sh.stop != 0;
+}
+
+// ------------------------------------------------------------------ units
+// Units: shared-expert tiles j < nS, then routed tile (j - nS) % nI of slot
+// (j - nS) / nI.  CTA c takes j = c, c + grid, c + 2 grid, ...  Its steps:
+// the up of each unit and the down of each unit, ordered so that a unit's
+// down comes one unit after its up (the relu^2 rows are ready by then),
+// except that a shared first unit is followed by its own down at once (its
+// successors wait for the routing).
+struct Units {
+  int c, G, nS, nI, N;  // N = nS + U * nI, the units of the pass (known after routing)
+  __device__ __forceinline__ int count() const { return c < N ? (N - 1 - c) / G + 1 : 0; }
+  __device__ __forceinline__ int unit(int n) const { return c + n * G; }
+  __device__ __forceinline__ bool shared_first() const { return c < nS; }
+};
+
+// The s-th step of a CTA with m units: kind 0 = up, 1 = down, of its unit n.
+// m = 0 (routing not yet known) gives the steps that do not depend on it:
+// with a shared first unit, its up and its down.
+__device__ __forceinline__ bool step_of(const Units& u, int m, int s, int* kind, int* n) {
+  if (u.shared_first()) {
+    if (s == 0) { *kind = 0; *n = 0; return true; }
+    if (s == 1) { *kind = 1; *n = 0; return true; }
+    s -= 2;
+    // routed units 1 .. m-1: up(1), up(2), down(1), up(3), down(2), ..., down(m-1)
+    const int r = m - 1;
+    if (r <= 0) return false;
+    if (s == 0) { *kind = 0; *n = 1; return true; }
+    // after the first up: pairs (up(i + 1), down(i)) for i = 1 .. r - 1, then down(r)
+    const int q = s - 1;
+    const int i = 1 + q / 2;
+    if (i < r) {
+      *kind = (q & 1) ? 1 : 0;
+      *n = (q & 1) ? i : i + 1;
+      return true;
+    }
+    if (q == 2 * (r - 1)) { *kind = 1; *n = r; return true; }
+    return false;
+  }
+  // up(0), up(1), down(0), up(2), down(1), ..., down(m-1)
+  if (m <= 0) return false;
+  if (s == 0) { *kind = 0; *n = 0; return true; }
+  const int q = s - 1;
+  const int i = q / 2;
+  if (i < m - 1) {
+    *kind = (q & 1) ? 1 : 0;
+    *n = (q & 1) ? i : i + 1;
+    return true;
+  }
+  if (q == 2 * (m - 1)) { *kind = 1; *n = m - 1; return true; }
+  return false;
+}
+
+// ---------------------------------------------------------------- routing
+// Routing warps (rt 0..127).  One pass over the tokens, the norm weight and
+// this CTA's gate rows (blockIdx.x and, with E > grid, blockIdx.x + grid):
+// the sums of squares and the dot products G_e . (x_t * w) come out of the
+// same loads.  CTA 0 also writes the normed rows and the residual.
+template <int MAXT>
+__device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
+  const int H = p.H, T = p.T, E = p.E, G = gridDim.x;
+  const int nv = H / 8;
+  const int warp = rt >> 5, lane = rt & 31;
+  const int e0 = blockIdx.x, e1 = blockIdx.x + G;
+  const bool has0 = e0 < E, has1 = e1 < E;
+  // One or two tokens: every chunk's loads in flight first, the token chunks
+  // kept in registers for the normed rows below.  More tokens would spill
+  // those registers: their chunks are loaded one at a time, and again for
+  // the normed rows.
+  constexpr bool kHold = MAXT <= 2;
+  constexpr int kHeld = kHold ? kMaxChunks : 1;
+  uint4 xv[kHeld][MAXT], wv[kHeld];
+  auto load_chunk = [&](int j, uint4 (&x)[MAXT], uint4& w, uint4& a, uint4& b) {
+    const int c = rt + j * kRouteThreads;
+    const bool in = c < nv;
+    w = in ? __ldg(reinterpret_cast<const uint4*>(p.norm_w) + c) : make_uint4(0, 0, 0, 0);
+    a = in && has0 ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e0) * H) + c)
+                   : make_uint4(0, 0, 0, 0);
+    b = in && has1 ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e1) * H) + c)
+                   : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int t = 0; t < MAXT; ++t)
+      x[t] = in && t < T ? reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c]
+                         : make_uint4(0, 0, 0, 0);
+  };
+  float ss[MAXT], d0[MAXT], d1[MAXT];
+#pragma unroll
+  for (int t = 0; t < MAXT; ++t) ss[t] = d0[t] = d1[t] = 0.f;
+  auto accumulate = [&](const uint4 (&x)[MAXT], const uint4& wq, const uint4& aq,
+                        const uint4& bq) {
+    float w[8], a[8], b[8];
+    unpack8(wq, w);
+    unpack8(aq, a);
+    unpack8(bq, b);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      a[q] *= w[q];
+      b[q] *= w[q];
+    }
+#pragma unroll
+    for (int t = 0; t < MAXT; ++t) {
+      float f[8];
+      unpack8(x[t], f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        ss[t] += f[q] * f[q];
+        d0[t] += a[q] * f[q];
+        d1[t] += b[q] * f[q];
+      }
+    }
+  };
+  if constexpr (kHold) {
+    uint4 g0[kMaxChunks], g1[kMaxChunks];
+#pragma unroll
+    for (int j = 0; j < kMaxChunks; ++j) load_chunk(j, xv[j], wv[j], g0[j], g1[j]);
+#pragma unroll
+    for (int j = 0; j < kMaxChunks; ++j) accumulate(xv[j], wv[j], g0[j], g1[j]);
+  } else {
+#pragma unroll 1
+    for (int j = 0; j < kMaxChunks; ++j) {
+      uint4 g0, g1;
+      load_chunk(j, xv[0], wv[0], g0, g1);
+      accumulate(xv[0], wv[0], g0, g1);
+    }
+  }
+  if (rt < E) sh.bias[rt] = p.gate_bias ? p.gate_bias[rt] : 0.f;
+  if (rt + kRouteThreads < E)
+    sh.bias[rt + kRouteThreads] = p.gate_bias ? p.gate_bias[rt + kRouteThreads] : 0.f;
+#pragma unroll
+  for (int t = 0; t < MAXT; ++t) {
+    const float v0 = warp_sum(ss[t]), v1 = warp_sum(d0[t]), v2 = warp_sum(d1[t]);
+    if (lane == 0) {
+      sh.red[warp][t] = v0;
+      sh.red[warp][MAXT + t] = v1;
+      sh.red[warp][2 * MAXT + t] = v2;
+    }
+  }
+  named_barrier(kBarRoute, kRouteThreads);
+  // the routing loads have returned (their sums are in shared memory): the
+  // weight stream may start.  Routing decides when the routed weights can
+  // stream, so its loads go first.
+  if (rt == 0) mbar_arrive(&sh.loads_out);
+  if (rt < T) {
+    float s = 0.f, a = 0.f, b = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      s += sh.red[w][rt];
+      a += sh.red[w][MAXT + rt];
+      b += sh.red[w][2 * MAXT + rt];
+    }
+    const float r = rsqrtf(s / float(H) + p.eps);
+    sh.rs[rt] = r;
+    if (has0) p.ws.logits[rt * E + e0] = a * r;
+    if (has1) p.ws.logits[rt * E + e1] = b * r;
+  }
+  named_barrier(kBarRoute, kRouteThreads);
+  // this CTA's copy of the normed rows n = x * r * w (bf16), for its own
+  // TMA loads
+  bf16* x16 = p.ws.x16 + size_t(blockIdx.x) * kDecodeN * H;
+#pragma unroll
+  for (int j = 0; j < kMaxChunks; ++j) {
+    const int c = rt + j * kRouteThreads;
+    if (c < nv) {
+      const int hj = kHold ? j : 0;
+      if (!kHold) {
+        wv[0] = __ldg(reinterpret_cast<const uint4*>(p.norm_w) + c);
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t)
+          if (t < T) xv[0][t] = reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c];
+      }
+      float w[8];
+      unpack8(wv[hj], w);
+#pragma unroll
+      for (int t = 0; t < MAXT; ++t) {
+        if (t < T) {
+          float f[8];
+          unpack8(xv[hj][t], f);
+          const float r = sh.rs[t];
+          reinterpret_cast<uint4*>(x16 + size_t(t) * H)[c] =
+              make_uint4(pack_bf16x2(f[0] * r * w[0], f[1] * r * w[1]),
+                         pack_bf16x2(f[2] * r * w[2], f[3] * r * w[3]),
+                         pack_bf16x2(f[4] * r * w[4], f[5] * r * w[5]),
+                         pack_bf16x2(f[6] * r * w[6], f[7] * r * w[7]));
+        }
+      }
+    }
+  }
+  fence_proxy_async_global();
+  named_barrier(kBarRoute, kRouteThreads);
+  if (rt == 0) mbar_arrive(&sh.tokens);
+  if (blockIdx.x == 0) {  // the residual
+#pragma unroll
+    for (int j = 0; j < kMaxChunks; ++j) {
+      const int c = rt + j * kRouteThreads;
+      if (c < nv) {
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t)
+          if (t < T)
+            reinterpret_cast<uint4*>(p.residual + size_t(t) * H)[c] =
+                kHold ? xv[kHold ? j : 0][t]
+                      : reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c];
+      }
+    }
+  }
+  named_barrier(kBarRoute, kRouteThreads);
+  if (rt == 0) red_release_add(p.ws.sync + kRouteArrived, 1u);
+}
+
+// Once every CTA's logits are in: the sigmoid top-k of every token and the
+// routed slot table (identical in every CTA).  Returns false on timeout.
+__device__ bool route_select(const FusedParams& p, Shared& sh, int rt, volatile int* abort) {
+  const int T = p.T, E = p.E, k = p.k;
+  const int warp = rt >> 5, lane = rt & 31;
+  if (rt == 0) {
+    sh.route_fail = 0;
+    if (!wait_counter(p.ws.sync + kRouteArrived, gridDim.x, abort)) {
+      record_timeout(p.status, abort);
+      sh.route_fail = 1;
+    }
+  }
+  named_barrier(kBarRoute, kRouteThreads);
+  if (sh.route_fail) return false;
+  for (int t = warp; t < T; t += 4)
+    warp_topk(p.ws.logits + t * E, p.gate_bias ? sh.bias : nullptr, E, k, p.rsf,
+              sh.sel_idx + t * k, sh.sel_w + t * k);
+  for (int i = rt; i < kMaxSlots * kDecodeN; i += kRouteThreads) (&sh.seg_w[0][0])[i] = 0.f;
+  named_barrier(kBarRoute, kRouteThreads);
+  const int R = T * k;
+  for (int f = rt; f < R; f += kRouteThreads) {
+    const int e = sh.sel_idx[f];
+    int first = 1;
+    for (int g = 0; g < f; ++g) first &= sh.sel_idx[g] != e;
+    sh.first_use[f] = first;
+    if (blockIdx.x == 0) {  // the routing of the pass, for moe_copy_routing
+      p.ws.idx[f] = e;
+      p.ws.w[f] = sh.sel_w[f];
+    }
+  }
+  named_barrier(kBarRoute, kRouteThreads);
+  if (warp == 0) {  // exclusive scan of the first-use flags (R <= 128)
+    int base = 0;
+    for (int f0 = 0; f0 < R; f0 += 32) {
+      const int f = f0 + lane;
+      const int v = f < R ? sh.first_use[f] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (v) {
+        const int e = sh.sel_idx[f];
+        if (unsigned(e) < unsigned(E)) sh.slot_of[e] = base + incl - 1;
+        sh.seg_expert[base + incl - 1] = e;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) sh.U = base;
+  }
+  named_barrier(kBarRoute, kRouteThreads);
+  for (int f = rt; f < R; f += kRouteThreads) {
+    const int e = sh.sel_idx[f];
+    if (unsigned(e) < unsigned(E)) sh.seg_w[sh.slot_of[e]][f / k] = sh.sel_w[f];
+  }
+  // an id outside [0, E) (only from NaN logits) is routed nowhere
+  for (int s = rt; s < sh.U; s += kRouteThreads)
+    if (unsigned(sh.seg_expert[s]) >= unsigned(E)) {
+      sh.seg_expert[s] = 0;
+      atomicOr(p.status, kStatusBadIndex);
+    }
+  named_barrier(kBarRoute, kRouteThreads);
+  return true;
+}
+
+
+// ------------------------------------------------------------- epilogue
+// The relu^2 rows of a unit go into a shared-memory buffer laid out exactly
+// as a TMA box of the token operand would be (16 token rows x 64 K per 2 KB
+// chunk, 128-byte swizzle: the 16-byte chunk j of row t sits at j ^ (t % 8)),
+// so the down MMA reads it with the usual descriptor.
+__device__ __forceinline__ void store_u_row(uint8_t* ubuf, int rloc, const float (&v)[kDecodeN]) {
+  const int kk = rloc >> 6, k = rloc & 63;
+  uint8_t* base = ubuf + kk * kBBytes + (k & 7) * 2;
+#pragma unroll
+  for (int t = 0; t < kDecodeN; ++t)
+    *reinterpret_cast<bf16*>(base + t * 128 + ((((k >> 3) ^ (t & 7)) & 7) << 4)) =
+        __float2bfloat16_rn(v[t]);
+}
+
+// Unit n of CTA c: shared tile j < nS, or routed tile (j - nS) % nI of slot
+// (j - nS) / nI.
+struct UnitInfo {
+  bool shared;
+  int slot, expert, row0, rows;  // rows: valid intermediate rows of the weight matrix (S or I)
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const FusedParams& p, const Shared& sh,
+                                              const Units& u, int n) {
+  UnitInfo f;
+  const int j = u.unit(n);
+  f.shared = j < u.nS;
+  if (f.shared) {
+    f.slot = -1;
+    f.expert = 0;
+    f.row0 = j * kBM;
+    f.rows = p.S;
+  } else {
+    const int r = j - u.nS;
+    f.slot = r / u.nI;
+    f.expert = sh.seg_expert[f.slot];
+    f.row0 = (r - f.slot * u.nI) * kBM;
+    f.rows = p.I;
+  }
+  return f;
+}
+
+// 64-wide k-blocks of a unit's down slice that hold weights (the last tile
+// of an expert may have only 64 valid rows).
+__device__ __forceinline__ int down_kk(const UnitInfo& f) { return f.rows - f.row0 >= kBM ? 2 : 1; }
+
+// ---------------------------------------------------------------- kernel
+template <int MAXT>
+__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ FusedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* tiles = smem_raw + pad;
+  uint8_t* ubufs = tiles + kStages * kStageBytes;  // two relu^2 row buffers
+  Shared& sh = *reinterpret_cast<Shared*>(ubufs + 2 * kUBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int nH = (p.H + kBM - 1) / kBM;
+  const int kbH = p.H / 64;
+
+  Units un;
+  un.c = cta;
+  un.G = G;
+  un.nS = (p.S + kBM - 1) / kBM;
+  un.nI = (p.I + kBM - 1) / kBM;
+  un.N = un.nS;  // the routed units are added once the routing is known
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.tfull[b], 1);
+      mbar_init(&sh.tempty[b], 4);
+      mbar_init(&sh.ufull[b], 1);
+      mbar_init(&sh.ufree[b], 1);
+    }
+    mbar_init(&sh.down_done, 1);
+    mbar_init(&sh.loads_out, 1);
+    mbar_init(&sh.tokens, 1);
+    mbar_init(&sh.routed, 1);
+    mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    sh.U = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tm_up);
+    tma_prefetch_desc(&p.tm_sup);
+    tma_prefetch_desc(&p.tm_down);
+    tma_prefetch_desc(&p.tm_sdown);
+    tma_prefetch_desc(&p.tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sh.tmem_base;
+  volatile int* abort = &sh.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      // The up GEMM's token rows (this CTA's normed rows) are written by the
+      // routing warps; until then those B loads wait in a queue (issue
+      // order) while the weight loads go out.
+      struct PendB {
+        int stage, x;
+      };
+      PendB pend[kStages] = {};
+      int npend = 0;
+      bool tok_ready = false;
+      const int xrow = cta * kDecodeN;
+      auto flush = [&](bool force) {
+        if (!tok_ready && mbar_test_wait(&sh.tokens, 0)) {
+          tok_ready = true;
+          fence_proxy_async_global();
+        }
+        if (!tok_ready && !force) return;
+        for (int j = 0; j < npend; ++j)
+          tma_load_2d(tiles + pend[j].stage * kStageBytes + kABytes, &p.tm_x,
+                      &sh.full[pend[j].stage], pend[j].x, xrow);
+        npend = 0;
+      };
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      // the routing warps' loads go out first (the routing decides when the
+      // routed weights can stream)
+      if (!mbar_wait(&sh.loads_out, 0, abort)) {
+        record_timeout(p.status, abort);
+        ok = false;
+      }
+      // one weight box (+ token box for up) into the next free stage
+      auto issue = [&](const CUtensorMap* map, int ax, int ay, bool up, int bx) -> bool {
+        if (!mbar_test_wait(&sh.empty[stage], phase ^ 1u)) {
+          const long long t0 = clock64();
+          // try_wait suspends this thread (no issue slots taken from the
+          // other warps) when no token load is pending; with pending loads
+          // it polls the tokens barrier between short sleeps
+          while (npend ? !mbar_test_wait(&sh.empty[stage], phase ^ 1u)
+                       : !mbar_try_wait(&sh.empty[stage], phase ^ 1u)) {
+            if (npend) {
+              flush(false);
+              __nanosleep(64);
+            }
+            if (*abort || clock64() - t0 > kWaitLimitCycles) {
+              record_timeout(p.status, abort);
+              return false;
+            }
+          }
+        }
+        uint8_t* sa = tiles + stage * kStageBytes;
+        mbar_arrive_expect_tx(&sh.full[stage], up ? kStageBytes : kABytes);
+        tma_load_2d(sa, map, &sh.full[stage], ax, ay);
+        if (up) {
+          if (npend) flush(false);
+          if (tok_ready)
+            tma_load_2d(sa + kABytes, &p.tm_x, &sh.full[stage], bx, xrow);
+          else
+            pend[npend++] = PendB{stage, bx};
+        }
+        ++issued;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
+      int m = 0;
+      bool routed = false;
+      for (int s = 0; ok; ++s) {
+        int kind, n;
+        if (!step_of(un, m, s, &kind, &n)) {
+          if (routed) break;
+          // the routed units: wait for this CTA's routing (test_wait: the
+          // pending token loads are this thread's to issue)
+          const long long t0 = clock64();
+          while (npend ? !mbar_test_wait(&sh.routed, 0) : !mbar_try_wait(&sh.routed, 0)) {
+            if (npend) {
+              flush(false);
+              __nanosleep(64);
+            }
+            if (*abort || clock64() - t0 > kWaitLimitCycles) {
+              ok = false;
+              break;
+            }
+          }
+          if (!ok || *abort) {
+            record_timeout(p.status, abort);
+            ok = false;
+            break;
+          }
+          routed = true;
+          un.N = un.nS + sh.U * un.nI;
+          m = un.count();
+          if (!step_of(un, m, s, &kind, &n)) break;
+        }
+        const UnitInfo f = unit_info(p, sh, un, n);
+        if (kind == 0) {  // up: W_up[rows] x tokens, K = H
+          const CUtensorMap* map = f.shared ? &p.tm_sup : &p.tm_up;
+          const int ay = f.shared ? f.row0 : f.expert * p.I + f.row0;
+          for (int kb = 0; ok && kb < kbH; ++kb) ok = issue(map, kb * 64, ay, true, kb * 64);
+        } else {  // down: W_down[:, rows] for every 128-row block of H
+          const CUtensorMap* map = f.shared ? &p.tm_sdown : &p.tm_down;
+          const int nkk = down_kk(f);
+          for (int r = 0; ok && r < nH; ++r) {
+            const int ay = (f.shared ? 0 : f.expert * p.H) + r * kBM;
+            for (int kk = 0; ok && kk < nkk; ++kk) ok = issue(map, f.row0 + kk * 64, ay, false, 0);
+          }
+        }
+      }
+      // the remaining token loads (also on an abort, so that every issued
+      // stage completes and can be drained)
+      if (ok && npend) {
+        const long long t0 = clock64();
+        while (npend) {
+          flush(false);
+          if (npend && (*abort || clock64() - t0 > kWaitLimitCycles)) {
+            record_timeout(p.status, abort);
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (!ok) {
+        flush(true);
+        int s = stage;
+        uint32_t ph = phase;
+        const int n = issued < kStages ? issued : kStages;
+        for (int i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = kStages - 1;
+            ph ^= 1u;
+          }
+          int zero = 0;
+          mbar_wait(&sh.full[s], ph, &zero);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(kBM, kDecodeN, 1, 1);  // BF16 x BF16 -> F32
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int m = 0;
+      bool routed = false, any = false;
+      for (int s = 0; ok; ++s) {
+        int kind, n;
+        if (!step_of(un, m, s, &kind, &n)) {
+          if (routed) break;
+          if (!mbar_wait(&sh.routed, 0, abort) || *abort) {
+            record_timeout(p.status, abort);
+            ok = false;
+            break;
+          }
+          routed = true;
+          un.N = un.nS + sh.U * un.nI;
+          m = un.count();
+          if (!step_of(un, m, s, &kind, &n)) break;
+        }
+        const UnitInfo f = unit_info(p, sh, un, n);
+        const int b = n & 1;
+        const uint32_t par = (n >> 1) & 1;
+        any = true;
+        if (kind == 0) {
+          // up into accumulator b (free once the epilogue has read unit n - 2)
+          if (!mbar_wait(&sh.tempty[b], par ^ 1u, abort)) {
+            record_timeout(p.status, abort);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem_base + uint32_t(b * kDecodeN);
+          for (int kb = 0; kb < kbH; ++kb) {
+            if (!mbar_wait(&sh.full[stage], phase, abort)) {
+              record_timeout(p.status, abort);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint8_t* sa = tiles + stage * kStageBytes;
+            const uint64_t ad = smem_desc_sw128(sa);
+            const uint64_t bd = smem_desc_sw128(sa + kABytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t koff = uint64_t((kk * 32) >> 4);
+              umma_f16(d, ad + koff, bd + koff, idesc, (kb != 0 || kk != 0) ? 1u : 0u);
+            }
+            umma_commit(&sh.empty[stage]);
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (ok) umma_commit(&sh.tfull[b]);
+        } else {
+          // down: the unit's relu^2 rows (buffer b) against W_down[:, rows],
+          // added into the H x 16 accumulator
+          if (!mbar_wait(&sh.ufull[b], par, abort)) {
+            record_timeout(p.status, abort);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* ub = ubufs + b * kUBytes;
+          const int nkk = down_kk(f);
+          for (int r = 0; ok && r < nH; ++r) {
+            const uint32_t d = tmem_base + uint32_t((2 + r) * kDecodeN);
+            for (int kc = 0; kc < nkk; ++kc) {
+              if (!mbar_wait(&sh.full[stage], phase, abort)) {
+                record_timeout(p.status, abort);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t ad = smem_desc_sw128(tiles + stage * kStageBytes);
+              const uint64_t bd = smem_desc_sw128(ub + kc * kBBytes);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t koff = uint64_t((kk * 32) >> 4);
+                umma_f16(d, ad + koff, bd + koff, idesc, (n != 0 || kc != 0 || kk != 0) ? 1u : 0u);
+              }
+              umma_commit(&sh.empty[stage]);
+              if (++stage == kStages) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+          }
+          if (ok) umma_commit(&sh.ufree[b]);
+        }
+      }
+      if (ok && any) umma_commit(&sh.down_done);
+      umma_commit(&sh.drain);
+      int zero = 0;
+      mbar_wait(&sh.drain, 0, &zero);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int tid = threadIdx.x - 64;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int rloc = q * 32 + lane;
+    const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
+    bool ok = true, routed = false;
+    int m = un.shared_first() ? 1 : 0;
+    for (int n = 0; ok; ++n) {
+      if (n >= m) {
+        if (routed) break;
+        // the routed units (and their routing weights): wait for the routing
+        if (lane == 0 && !mbar_wait(&sh.routed, 0, abort)) record_timeout(p.status, abort);
+        __syncwarp();
+        if (epi_stop(sh, tid)) {
+          ok = false;
+          break;
+        }
+        routed = true;
+        un.N = un.nS + sh.U * un.nI;
+        m = un.count();
+        if (n >= m) break;
+      }
+      const UnitInfo f = unit_info(p, sh, un, n);
+      const int b = n & 1;
+      const uint32_t par = (n >> 1) & 1;
+      // the up accumulator of unit n
+      if (lane == 0 && !mbar_wait(&sh.tfull[b], par, abort)) record_timeout(p.status, abort);
+      __syncwarp();
+      if (epi_stop(sh, tid)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(lane_base + uint32_t(b * kDecodeN), r);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tempty[b]);
+      // relu^2 times the routing weight (1 for the shared expert); rows past
+      // the matrix (an expert's last tile) and tokens past T are zero
+      float v[kDecodeN];
+      const bool valid = f.row0 + rloc < f.rows;
+#pragma unroll
+      for (int c = 0; c < kDecodeN; ++c) {
+        const float w = f.shared ? (c < p.T ? 1.f : 0.f) : sh.seg_w[f.slot][c];
+        const float a = __uint_as_float(r[c]);
+        v[c] = valid && w != 0.f ? (a > 0.f ? a * a : 0.f) * w : 0.f;
+      }
+      // buffer b is free once unit n - 2's down MMAs have completed
+      if (n >= 2) {
+        if (lane == 0 && !mbar_wait(&sh.ufree[b], ((n - 2) >> 1) & 1, abort))
+          record_timeout(p.status, abort);
+        __syncwarp();
+        if (epi_stop(sh, tid)) {
+          ok = false;
+          break;
+        }
+      }
+      store_u_row(ubufs + b * kUBytes, rloc, v);
+      fence_proxy_async_shared();  // generic writes -> tensor core reads
+      named_barrier(kBarEpi, kEpiThreads);
+      if (tid == 0) mbar_arrive(&sh.ufull[b]);
+    }
+    // this CTA's partial output: the H x 16 down accumulator, columns < MAXT
+    if (ok && m > 0) {
+      if (lane == 0 && !mbar_wait(&sh.down_done, 0, abort)) record_timeout(p.status, abort);
+      __syncwarp();
+      if (!epi_stop(sh, tid)) {
+        tc_fence_after();
+        float* part = p.ws.part + size_t(cta) * kDecodeMaxT * p.H;
+        for (int rt = 0; rt < nH; ++rt) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(lane_base + uint32_t((2 + rt) * kDecodeN), r);
+          tmem_ld_wait();
+          const int row = rt * kBM + rloc;
+          if (row < p.H) {
+#pragma unroll
+            for (int c = 0; c < MAXT; ++c) part[size_t(c) * p.H + row] = __uint_as_float(r[c]);
+          }
+        }
+        tc_fence_before();
+        named_barrier(kBarEpi, kEpiThreads);
+        if (tid == 0) red_release_add(p.ws.sync + kPartialsDone, 1u);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- routing
+    const int rt = threadIdx.x - 192;
+    route_logits<MAXT>(p, sh, rt);
+    route_select(p, sh, rt, abort);
+    if (rt == 0) mbar_arrive(&sh.routed);  // (also on failure: the waiters then see abort)
+  }
+
+  // ----------------------------------------------- reduction and wind down
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+  // Rows [r0, r0 + nr) of the output: the partials of every CTA that had
+  // units, added in CTA order, plus the input row.  Once every CTA's logits
+  // are in, no CTA reads hidden any more, so the rows can be overwritten.
+  // (every thread takes the unit count from the slot table: only some
+  // roles have updated their own copy of it)
+  const int n_units = un.nS + sh.U * un.nI;
+  if (threadIdx.x == 0 && !*abort) {
+    const unsigned active = unsigned(n_units < G ? n_units : G);
+    if (!wait_counter(p.ws.sync + kPartialsDone, active, abort) ||
+        !wait_counter(p.ws.sync + kRouteArrived, unsigned(G), abort))
+      record_timeout(p.status, abort);
+  }
+  __syncthreads();
+  if (!*abort) {
+    const int T = p.T, H = p.H;
+    const int active = n_units < G ? n_units : G;
+    const int R0 = (H + G - 1) / G;
+    const int r0 = cta * R0;
+    const int nr = min(H, r0 + R0) - r0;
+    if (nr > 0) {
+      // stage every partial value of the slice in shared memory (the ring
+      // is idle now), [source CTA][token][row]
+      float* stage_f = reinterpret_cast<float*>(tiles);
+      const int per = T * nr;
+      const int count = active * per;
+      for (int i = threadIdx.x; i < count; i += kThreads) {
+        const int src = i / per, rem = i - src * per;
+        const int t = rem / nr, row = rem - t * nr;
+        stage_f[i] = __ldcg(p.ws.part + (size_t(src) * kDecodeMaxT + t) * H + r0 + row);
+      }
+      __syncthreads();
+      // each output is summed by kParts threads over fixed, consecutive
+      // source ranges, then the kParts sums in order: a fixed order
+      constexpr int kParts = 8;
+      float* sums = stage_f + count;  // [per][kParts]
+      const int span = (active + kParts - 1) / kParts;
+      for (int i = threadIdx.x; i < per * kParts; i += kThreads) {
+        const int o = i / kParts, part = i - o * kParts;
+        const int s0 = part * span, s1 = min(active, s0 + span);
+        float acc = 0.f;
+        for (int src = s0; src < s1; ++src) acc += stage_f[src * per + o];
+        sums[i] = acc;
+      }
+      __syncthreads();
+      for (int o = threadIdx.x; o < per; o += kThreads) {
+        const int t = o / nr, row = r0 + (o - t * nr);
+        float acc = 0.f;
+#pragma unroll
+        for (int part = 0; part < kParts; ++part) acc += sums[o * kParts + part];
+        const size_t at = size_t(t) * H + row;
+        p.out[at] = __float2bfloat16_rn(__bfloat162float(p.hidden[at]) + acc);
+      }
+    }
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA out resets the launch's synchronisation words: every
+    // other CTA has passed its last wait on them
+    __threadfence();
+    sh.flag = atomicAdd(p.ws.sync + kExited, 1u) == unsigned(G - 1);
+    if (sh.flag) {
+      p.ws.sync[kRouteArrived] = 0u;
+      p.ws.sync[kPartialsDone] = 0u;
+      p.ws.sync[kExited] = 0u;
+    }
+  }
+}
+
+}  // namespace
+
+bool fused_decode_supported(const moe_config& c) {
+  // the routing warps hold a token row in kMaxChunks 8-element chunks each;
+  // the H x 16 down accumulator fits next to the two up accumulators in TMEM
+  return c.latent_size == 0 && c.expert_wdtype == MOE_WEIGHTS_BF16 &&
+         c.shared_wdtype == MOE_WEIGHTS_BF16 &&
+         c.hidden_size <= kMaxChunks * kRouteThreads * 8 &&
+         (c.hidden_size + kBM - 1) / kBM <= kMaxRowTiles;
+}
+
+cudaError_t prepare_fused_decode() {
+  const int bytes = kSmem + int(sizeof(Shared));
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(decode_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                bytes)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(decode_fused_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                bytes)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(decode_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                bytes)) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(decode_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              bytes);
+}
+
+cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
+  const moe_config& c = *a.cfg;
+  FusedParams p;
+  p.tm_up = *a.tm_up;
+  p.tm_sup = *a.tm_sup;
+  p.tm_down = *a.tm_down;
+  p.tm_sdown = *a.tm_sdown;
+  p.tm_x = *a.tm_x;
+  p.hidden = a.hidden;
+  p.residual = a.residual;
+  p.out = a.hidden;
+  p.norm_w = static_cast<const bf16*>(a.w->norm_w);
+  p.gate_w = static_cast<const bf16*>(a.w->gate_w);
+  p.gate_bias = a.w->gate_bias;
+  p.T = a.T;
+  p.H = c.hidden_size;
+  p.E = c.num_experts;
+  p.k = c.top_k;
+  p.I = c.moe_inter;
+  p.S = c.shared_inter;
+  p.eps = c.rms_eps;
+  p.rsf = c.routed_scaling_factor;
+  p.ws = *a.ws;
+  p.status = a.status;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem + sizeof(Shared);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.T <= 1) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<1>, p);
+  if (a.T <= 2) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<2>, p);
+  if (a.T <= 4) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<4>, p);
+  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<8>, p);
+}
+
+}  // namespace moe

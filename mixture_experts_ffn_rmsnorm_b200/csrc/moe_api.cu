@@ -82,7 +82,10 @@ struct moe_handle {
   int device;
   int num_sms;
   int D;           // routed-expert width
-  bool fp8;
+  bool fp8;         // routed experts E4M3
+  bool shared_fp8;  // shared expert E4M3
+  bool latent_fp8;  // fc1 / fc2 E4M3
+  bool need_nq;     // some GEMM reads the E4M3 copy of the normed tokens
   int gate_bn;     // router GEMM tile width (>= E)
   int last_launches;
   void* const* stage_events;  // profiling: caller-owned cudaEvent_t array
@@ -120,7 +123,12 @@ struct moe_handle {
   unsigned* u_amax;  // [Rm]      running row max of relu^2(up) (float bits)
   uint8_t* uq;       // [Rm, I]   E4M3 relu^2(up)
   float* u_scale;    // [Rm]
-  moe::DecodeWorkspace dec;
+  unsigned* v_amax;  // [Tm]      FP8 shared expert: running row max of relu^2(up)
+  uint8_t* vq;       // [Tm, S]   E4M3 shared relu^2(up)
+  float* v_scale;    // [Tm]
+  uint8_t* mq;       // [Tm, L]   FP8 fc2: E4M3 latent weighted sum
+  float* m_scale;    // [Tm]
+  moe::FusedWorkspace dec;
   // tensor maps
   CUtensorMap tm_gate_a, tm_gate_b, tm_fc1_a, tm_fc1_b;
   CUtensorMap tm_up_a, tm_up_b, tm_sup_a, tm_sup_b;
@@ -130,7 +138,7 @@ struct moe_handle {
   CUtensorMap tm_up_w, tm_sup_w, tm_down_w, tm_sdown_w;
   int up_bn, down_bn;
   CUtensorMap tm_fc2_a, tm_fc2_b;
-  CUtensorMap tm_dec_x, tm_dec_ub, tm_dec_vb;  // decode B operands (16-row boxes)
+  CUtensorMap tm_dec_x;  // decode token rows, one 16-row block per CTA (16-row boxes)
 };
 
 namespace {
@@ -162,7 +170,12 @@ moe_status validate_config(const moe_config* c) {
   if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps) ||
       !std::isfinite(c->routed_scaling_factor))
     return MOE_ERR_INVALID_CONFIG;
-  if (c->expert_wdtype != MOE_WEIGHTS_BF16 && c->expert_wdtype != MOE_WEIGHTS_FP8_E4M3_ROWSCALE)
+  for (int32_t dt : {c->expert_wdtype, c->shared_wdtype, c->latent_wdtype})
+    if (dt != MOE_WEIGHTS_BF16 && dt != MOE_WEIGHTS_FP8_E4M3_ROWSCALE)
+      return MOE_ERR_INVALID_CONFIG;
+  // FP8 routed experts are wired for the direct layer (their input rows are
+  // the E4M3 normed tokens)
+  if (c->expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE && c->latent_size > 0)
     return MOE_ERR_INVALID_CONFIG;
   // row counts of the stacked expert maps and tile tables must fit in int32
   const long long D = c->latent_size ? c->latent_size : c->hidden_size;
@@ -180,9 +193,16 @@ moe_status validate_weights(const moe_config* c, const moe_weights* w) {
   for (const void* p : req)
     if (!p) return MOE_ERR_NULL_POINTER;
   if (fp8 && (!w->up_scale || !w->down_scale)) return MOE_ERR_NULL_POINTER;
+  if (c->shared_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE &&
+      (!w->shared_up_scale || !w->shared_down_scale))
+    return MOE_ERR_NULL_POINTER;
   if (c->latent_size > 0 && (!w->fc1_w || !w->fc2_w)) return MOE_ERR_NULL_POINTER;
+  if (c->latent_size > 0 && c->latent_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE &&
+      (!w->fc1_scale || !w->fc2_scale))
+    return MOE_ERR_NULL_POINTER;
   const void* all[] = {w->norm_w, w->gate_w, w->gate_bias, w->up_w, w->down_w, w->up_scale,
-                       w->down_scale, w->shared_up_w, w->shared_down_w, w->fc1_w, w->fc2_w};
+                       w->down_scale, w->shared_up_w, w->shared_down_w, w->fc1_w, w->fc2_w,
+                       w->shared_up_scale, w->shared_down_scale, w->fc1_scale, w->fc2_scale};
   for (const void* p : all)
     if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
   return MOE_OK;
@@ -225,15 +245,26 @@ void carve(moe_handle* h, char* base) {
   h->m = L ? cv.take<bf16>(Tm * L) : nullptr;
   h->stage_h = cv.take<bf16>(Tm * H);
   h->stage_r = cv.take<bf16>(Tm * H);
-  if (h->fp8) {
+  if (h->need_nq) {
     h->nq = cv.take<uint8_t>(Tm * H);
     h->nq_scale = cv.take<float>(Tm);
+  }
+  if (h->fp8) {
     h->xs_scale = cv.take<float>(Rm);
     h->u_amax = cv.take<unsigned>(Rm);
     h->uq = cv.take<uint8_t>(Rm * I);
     h->u_scale = cv.take<float>(Rm);
   }
-  moe::carve_decode(&h->dec, c, h->num_sms, [&](size_t bytes) { return cv.take<char>(bytes); });
+  if (h->shared_fp8) {
+    h->v_amax = cv.take<unsigned>(Tm);
+    h->vq = cv.take<uint8_t>(Tm * S);
+    h->v_scale = cv.take<float>(Tm);
+  }
+  if (L && h->latent_fp8) {
+    h->mq = cv.take<uint8_t>(Tm * L);
+    h->m_scale = cv.take<float>(Tm);
+  }
+  moe::carve_fused(&h->dec, c, h->num_sms, [&](size_t bytes) { return cv.take<char>(bytes); });
   h->ws_bytes = cv.off;
 }
 
@@ -242,42 +273,48 @@ bool build_maps(moe_handle* h) {
   const uint64_t Tm = c.max_tokens, E = c.num_experts, H = c.hidden_size;
   const uint64_t Rm = Tm * c.top_k, D = h->D, I = c.moe_inter, S = c.shared_inter,
                  L = c.latent_size;
-  const bool f8 = h->fp8;
-  const uint64_t eb = f8 ? 1 : 2;  // bytes per routed-expert operand element
+  const bool f8 = h->fp8, sf8 = h->shared_fp8, lf8 = h->latent_fp8;
+  const uint64_t eb = f8 ? 1 : 2;   // bytes per routed-expert operand element
+  const uint64_t sb = sf8 ? 1 : 2;  // shared expert
+  const uint64_t lb = lf8 ? 1 : 2;  // fc1 / fc2
   bool ok = true;
   // router: A = [hi | lo] (K = 2H), B = gate [E, H] (k wraps at H)
   ok &= make_map(&h->tm_gate_a, h->gate_a, false, 2 * H, Tm, 2 * H * 2, moe::kBM);
   ok &= make_map(&h->tm_gate_b, h->w.gate_w, false, H, E, H * 2, h->gate_bn);
-  if (L) {
-    ok &= make_map(&h->tm_fc1_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
-    ok &= make_map(&h->tm_fc1_b, h->w.fc1_w, false, H, L, H * 2, h->gate_bn);
-    ok &= make_map(&h->tm_fc2_a, h->m, false, L, Tm, L * 2, moe::kBM);
-    ok &= make_map(&h->tm_fc2_b, h->w.fc2_w, false, L, H, L * 2, 128);
+  if (L) {  // FP8 fc1 / fc2 read the E4M3 normed tokens / latent sums
+    if (lf8)
+      ok &= make_map(&h->tm_fc1_a, h->nq, true, H, Tm, H, moe::kBM);
+    else
+      ok &= make_map(&h->tm_fc1_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
+    ok &= make_map(&h->tm_fc1_b, h->w.fc1_w, lf8, H, L, H * lb, h->gate_bn);
+    ok &= make_map(&h->tm_fc2_a, lf8 ? static_cast<const void*>(h->mq) : h->m, lf8, L, Tm,
+                   L * lb, moe::kBM);
+    ok &= make_map(&h->tm_fc2_b, h->w.fc2_w, lf8, L, H, L * lb, 128);
   }
   // grouped up: routed A = xs [Rm, D], B = up [E*I, D]; shared A = normed, B = [S, H]
   ok &= make_map(&h->tm_up_a, h->xs, f8, D, Rm, D * eb, moe::kBM);
   ok &= make_map(&h->tm_up_b, h->w.up_w, f8, D, E * I, D * eb, 128);
-  ok &= make_map(&h->tm_sup_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
-  ok &= make_map(&h->tm_sup_b, h->w.shared_up_w, false, H, S, H * 2, 128);
+  if (sf8)
+    ok &= make_map(&h->tm_sup_a, h->nq, true, H, Tm, H, moe::kBM);
+  else
+    ok &= make_map(&h->tm_sup_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
+  ok &= make_map(&h->tm_sup_b, h->w.shared_up_w, sf8, H, S, H * sb, 128);
   // grouped down: routed A = u [Rm, I], B = down [E*D, I]; shared A = v, B = [H, S]
   ok &= make_map(&h->tm_down_a, f8 ? static_cast<const void*>(h->uq) : h->u, f8, I, Rm, I * eb,
                  moe::kBM);
   ok &= make_map(&h->tm_down_b, h->w.down_w, f8, I, E * D, I * eb, 128);
-  ok &= make_map(&h->tm_sdown_a, h->v, false, S, Tm, S * 2, moe::kBM);
-  ok &= make_map(&h->tm_sdown_b, h->w.shared_down_w, false, S, H, S * 2, 128);
+  ok &= make_map(&h->tm_sdown_a, sf8 ? static_cast<const void*>(h->vq) : h->v, sf8, S, Tm,
+                 S * sb, moe::kBM);
+  ok &= make_map(&h->tm_sdown_b, h->w.shared_down_w, sf8, S, H, S * sb, 128);
   h->up_bn = prefill_bn(I, S);
   h->down_bn = prefill_bn(D, H);
   ok &= make_map(&h->tm_up_w, h->w.up_w, f8, D, E * I, D * eb, h->up_bn);
-  ok &= make_map(&h->tm_sup_w, h->w.shared_up_w, false, H, S, H * 2, h->up_bn);
+  ok &= make_map(&h->tm_sup_w, h->w.shared_up_w, sf8, H, S, H * sb, h->up_bn);
   ok &= make_map(&h->tm_down_w, h->w.down_w, f8, I, E * D, I * eb, h->down_bn);
-  ok &= make_map(&h->tm_sdown_w, h->w.shared_down_w, false, S, H, S * 2, h->down_bn);
-  if (moe::decode_supported(c)) {
-    const uint64_t U = moe::decode_max_slots(c);
-    ok &= make_map(&h->tm_dec_x, h->dec.x16, false, H, moe::kDecodeN, H * 2, moe::kDecodeN);
-    ok &= make_map(&h->tm_dec_ub, h->dec.ub, false, I, (U + 1) * moe::kDecodeN, I * 2,
-                   moe::kDecodeN);
-    ok &= make_map(&h->tm_dec_vb, h->dec.vb, false, S, moe::kDecodeN, S * 2, moe::kDecodeN);
-  }
+  ok &= make_map(&h->tm_sdown_w, h->w.shared_down_w, sf8, S, H, S * sb, h->down_bn);
+  if (moe::fused_decode_supported(c))
+    ok &= make_map(&h->tm_dec_x, h->dec.x16, false, H, uint64_t(h->num_sms) * moe::kDecodeN,
+                   H * 2, moe::kDecodeN);
   return ok;
 }
 
@@ -323,6 +360,11 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
     p.tmB[1] = h->tm_fc1_b;
     p.cls[1] = dense_class(c.hidden_size, c.latent_size, T, moe::EPI_BF16, h->z, c.latent_size,
                            h->gate_bn);
+    if (h->latent_fp8) {  // W8A8: acc * token scale * weight-row scale
+      p.cls[1].fp8 = 1;
+      p.cls[1].row_scale = h->nq_scale;
+      p.cls[1].col_scale = h->w.fc1_scale;
+    }
     p.nclasses = 2;
   }
   const int mt = p.cls[0].mtiles;
@@ -335,7 +377,7 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
       // With LatentMoE fc1 in the launch, cut the router tiles (K = 2H) into
       // pieces of at most half fc1's K, so that no router tile is the
       // launch's long pole (more pieces when idle SMs allow).
-      const int nko = (p.cls[1].K + 63) / 64;
+      const int nko = (p.cls[1].K + (p.cls[1].fp8 ? 127 : 63)) / (p.cls[1].fp8 ? 128 : 64);
       const int cut = 2 * ((nk + nko - 1) / nko);
       if (ks < cut) ks = cut;
     }
@@ -347,7 +389,7 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
   }
   p.cls[0].ksplit = ks;
   MOE_TRY(moe::launch_rmsnorm(hidden, static_cast<const bf16*>(h->w.norm_w), residual, h->gate_a,
-                              h->fp8 && with_fc1 ? h->nq : nullptr, h->nq_scale, T,
+                              h->need_nq && with_fc1 ? h->nq : nullptr, h->nq_scale, T,
                               c.hidden_size, c.rms_eps, ks > 1 ? h->expert_hist : nullptr,
                               mt * c.num_experts, st));
   log->done(st);
@@ -410,6 +452,12 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.tmA[1] = h->tm_sup_a;
   p.tmB[1] = h->tm_sup_w;
   p.cls[1] = dense_class(H, S, T, moe::EPI_RELU2_BF16, h->v, S, h->up_bn);
+  if (h->shared_fp8) {  // W8A8, row max of relu^2 for requantisation
+    p.cls[1].fp8 = 1;
+    p.cls[1].row_scale = h->nq_scale;
+    p.cls[1].col_scale = h->w.shared_up_scale;
+    p.cls[1].row_amax = h->v_amax;
+  }
   p.nclasses = 2;
   p.tile_table = h->tiles;
   p.n_mtiles = h->n_mtiles;
@@ -419,8 +467,11 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   MOE_TRY(moe::launch_grouped_gemm(p, h->up_bn, h->num_sms, st));
   log->done(st);
 
-  if (h->fp8) {
-    MOE_TRY(moe::launch_quantize_rows(h->u, h->u_amax, h->uq, h->u_scale, R, I, st));
+  if (h->fp8 || h->shared_fp8) {  // E4M3 rows of relu^2(up), one scale per row
+    MOE_TRY(moe::launch_quantize_rows(h->fp8 ? h->u : nullptr, h->u_amax, h->uq, h->u_scale,
+                                      h->fp8 ? R : 0, I, h->shared_fp8 ? h->v : nullptr,
+                                      h->v_amax, h->vq, h->v_scale, h->shared_fp8 ? T : 0, S,
+                                      st));
     log->done(st);
   }
 
@@ -436,6 +487,12 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   p.tmA[1] = h->tm_sdown_a;
   p.tmB[1] = h->tm_sdown_w;
   p.cls[1] = dense_class(S, H, T, moe::EPI_F32, h->s, H, h->down_bn);
+  if (h->shared_fp8) {
+    p.cls[1].fp8 = 1;
+    p.cls[1].row_scale = h->v_scale;
+    p.cls[1].col_scale = h->w.shared_down_scale;
+    p.cls[1].row_amax = nullptr;
+  }
   p.sched = h->sched + 2;
   MOE_TRY(moe::launch_grouped_gemm(p, h->down_bn, h->num_sms, st));
   log->done(st);
@@ -445,13 +502,19 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
     log->done(st);
     return MOE_OK;
   }
-  MOE_TRY(moe::launch_latent_reduce(h->y, h->inv, h->wts, h->m, T, k, L, st));
+  MOE_TRY(moe::launch_latent_reduce(h->y, h->inv, h->wts, h->m, h->latent_fp8 ? h->mq : nullptr,
+                                    h->m_scale, T, k, L, st));
   log->done(st);
   GemmParams q;
   std::memset(&q, 0, sizeof(q));
   q.tmA[0] = h->tm_fc2_a;
   q.tmB[0] = h->tm_fc2_b;
   q.cls[0] = dense_class(L, H, T, moe::EPI_BLEND, hidden, H, 128);
+  if (h->latent_fp8) {
+    q.cls[0].fp8 = 1;
+    q.cls[0].row_scale = h->m_scale;
+    q.cls[0].col_scale = h->w.fc2_scale;
+  }
   q.nclasses = 1;
   q.blend_s = h->s;
   q.blend_res = residual;
@@ -462,68 +525,28 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
   return MOE_OK;
 }
 
-// Decode path (T <= 8): CUDA-core routing kernel, then two tcgen05 launches
-// with the weights as the 128-row operand and the tokens as N = 16, all
-// chained with programmatic dependent launch.
+// Decode path (T <= 8): one cooperative launch (decode_fused.cu) with the
+// weights as the 128-row operand and the tokens as N = 16.
 moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cudaStream_t st,
                           moe::LaunchLog* log) {
   const moe_config& c = h->cfg;
-  if (!moe::decode_supported(c) || T < 1 || T > MOE_DECODE_MAX_TOKENS)
+  if (!moe::fused_decode_supported(c) || T < 1 || T > MOE_DECODE_MAX_TOKENS)
     return MOE_ERR_INVALID_CONFIG;
-  const int H = c.hidden_size, I = c.moe_inter, S = c.shared_inter;
-  moe::DecodeRouteArgs ra;
-  ra.cfg = &c;
-  ra.w = &h->w;
-  ra.ws = &h->dec;
-  ra.hidden = hidden;
-  ra.residual = residual;
-  ra.T = T;
-  MOE_TRY(moe::launch_decode_route(ra, st));
-  log->done(st);
-
-  GemmParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.tmA[0] = h->tm_up_b;    // routed up weights [E*I, H] as the 128-row operand
-  p.tmB[0] = h->tm_dec_x;   // tokens [16, H]
-  p.tmA[1] = h->tm_sup_b;   // shared up weights [S, H]
-  p.tmB[1] = h->tm_dec_x;
-  p.cls[0] = dense_class(H, moe::kDecodeN, 0, moe::EPI_DEC_UP, nullptr, 0, moe::kDecodeN);
-  p.cls[1] = dense_class(H, moe::kDecodeN, 0, moe::EPI_DEC_UP, nullptr, 0, moe::kDecodeN);
-  p.nclasses = 2;
-  p.dec_tiles = h->dec.tiles_up;
-  p.dec_count = h->dec.n_tiles_up;
-  p.dec.T = T;
-  p.dec.M[0] = I;
-  p.dec.M[1] = S;
-  p.dec.n_first = (S + moe::kBM - 1) / moe::kBM;  // shared tiles lead the list
-  p.dec.seg_w = h->dec.seg_w;
-  p.dec.out_up[0] = h->dec.ub;
-  p.dec.out_up[1] = h->dec.vb;
-  p.dec.up_part = h->dec.up_part;
-  p.dec.up_counter = h->dec.up_counter;
-  p.status = h->status;
-  MOE_TRY(moe::launch_grouped_gemm(p, moe::kDecodeN, h->num_sms, st, true));
-  log->done(st);
-
-  p.tmA[0] = h->tm_down_b;   // routed down weights [E*H, I]
-  p.tmB[0] = h->tm_dec_ub;   // w * relu^2(up) per segment [(U+1)*16, I]
-  p.tmA[1] = h->tm_sdown_b;  // shared down weights [H, S]
-  p.tmB[1] = h->tm_dec_vb;   // [16, S]
-  p.cls[0] = dense_class(I, moe::kDecodeN, 0, moe::EPI_DEC_DOWN, nullptr, 0, moe::kDecodeN);
-  p.cls[1] = dense_class(S, moe::kDecodeN, 0, moe::EPI_DEC_DOWN, nullptr, 0, moe::kDecodeN);
-  p.dec_tiles = nullptr;
-  p.dec_count = h->dec.n_segments;  // output tiles over the concatenated segments
-  p.dec_concat = 1;
-  p.l2_prefetch[0] = p.l2_prefetch[1] = nullptr;
-  p.dec.M[0] = H;
-  p.dec.M[1] = H;
-  p.dec.seg_expert = h->dec.seg_expert;
-  p.dec.partial = h->dec.partial;
-  p.dec.mt_counter = h->dec.mt_counter;
-  p.dec.n_segments = h->dec.n_segments;
-  p.dec.residual = residual;
-  p.dec.hidden = hidden;
-  MOE_TRY(moe::launch_grouped_gemm(p, moe::kDecodeN, h->num_sms, st, true));
+  moe::FusedDecodeArgs a;
+  a.cfg = &c;
+  a.w = &h->w;
+  a.ws = &h->dec;
+  a.tm_up = &h->tm_up_b;      // routed up weights [E*I, H], 128-row boxes
+  a.tm_sup = &h->tm_sup_b;    // shared up weights [S, H]
+  a.tm_down = &h->tm_down_b;  // routed down weights [E*H, I]
+  a.tm_sdown = &h->tm_sdown_b;
+  a.tm_x = &h->tm_dec_x;
+  a.hidden = hidden;
+  a.residual = residual;
+  a.T = T;
+  a.grid = h->num_sms;
+  a.status = h->status;
+  MOE_TRY(moe::launch_fused_decode(a, st));
   log->done(st);
   return MOE_OK;
 }
@@ -571,11 +594,10 @@ moe_status moe_create(const moe_config* config, const moe_weights* weights, moe_
   h->num_sms = prop.multiProcessorCount;
   h->D = config->latent_size ? config->latent_size : config->hidden_size;
   h->fp8 = config->expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE;
+  h->shared_fp8 = config->shared_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE;
+  h->latent_fp8 = config->latent_size > 0 && config->latent_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE;
+  h->need_nq = (h->fp8 && config->latent_size == 0) || h->shared_fp8 || h->latent_fp8;
   h->gate_bn = config->num_experts <= 128 ? 128 : 256;
-  if (h->fp8 && config->latent_size > 0) {  // FP8 experts are wired for the direct layer
-    delete h;
-    return MOE_ERR_INVALID_CONFIG;
-  }
 
   carve(h, nullptr);
   void* ws = nullptr;
@@ -587,7 +609,7 @@ moe_status moe_create(const moe_config* config, const moe_weights* weights, moe_
   h->ws = ws;
   carve(h, static_cast<char*>(ws));
   if (cudaMemset(ws, 0, h->ws_bytes) != cudaSuccess || !build_maps(h) ||
-      moe::prepare_grouped_gemm() != cudaSuccess || moe::prepare_decode() != cudaSuccess) {
+      moe::prepare_grouped_gemm() != cudaSuccess || moe::prepare_fused_decode() != cudaSuccess) {
     cudaFree(ws);
     h->magic = 0;
     delete h;
@@ -629,7 +651,7 @@ moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t
   log.begin(s);
   const bool decode = path == MOE_PATH_DECODE ||
                       (path == MOE_PATH_AUTO && num_tokens <= MOE_DECODE_MAX_TOKENS &&
-                       moe::decode_supported(h->cfg));
+                       moe::fused_decode_supported(h->cfg));
   if (decode) {
     st = enqueue_decode(h, static_cast<bf16*>(hidden), static_cast<bf16*>(residual), num_tokens,
                         s, &log);
@@ -738,6 +760,13 @@ moe_status moe_get_device_status(moe_handle* h, int32_t* status, void* stream) {
   MOE_TRY(cudaMemcpyAsync(status, h->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
   MOE_TRY(cudaMemsetAsync(h->status, 0, sizeof(int32_t), s));
   MOE_TRY(cudaStreamSynchronize(s));
+  if (*status != 0) {
+    // A pass that gave up on a wait may have left its tile and schedule
+    // counters mid-count: start the next one from zero.
+    MOE_TRY(cudaMemsetAsync(h->dec.sync, 0, 4 * sizeof(unsigned), s));
+    MOE_TRY(cudaMemsetAsync(h->sched, 0, 4 * sizeof(int32_t), s));
+    MOE_TRY(cudaStreamSynchronize(s));
+  }
   return MOE_OK;
 }
 

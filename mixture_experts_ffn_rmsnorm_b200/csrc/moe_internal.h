@@ -195,14 +195,19 @@ cudaError_t launch_sort(const int* idx, const int* hist, int T, int k, int E, in
 cudaError_t launch_gather(const void* X, size_t ldx_bytes, const int* perm, int k, int R,
                           int row_bytes, void* xs, const float* scale, float* xs_scale,
                           cudaStream_t stream);
-// Per-row E4M3 quantisation of u [R, I] (bf16) with the row maxima amax
-// (float bits, reset to 0 afterwards): uq = sat(u / s), s = amax / 448.
-cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* amax, uint8_t* uq,
-                                 float* scale, int R, int I, cudaStream_t stream);
+// Per-row E4M3 quantisation of u [R, I] and v [Rv, S] (bf16) with their
+// row maxima (float bits, reset to 0 afterwards): q = sat(x / s),
+// s = amax / 448.  One launch for both sets (either may be empty).
+cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* u_amax, uint8_t* uq,
+                                 float* u_scale, int R, int I, const __nv_bfloat16* v,
+                                 unsigned* v_amax, uint8_t* vq, float* v_scale, int Rv, int S,
+                                 cudaStream_t stream);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* inv, const float* w,
                            const float* s, const __nv_bfloat16* residual,
                            __nv_bfloat16* hidden, int T, int k, int H, cudaStream_t stream);
+// mq / m_scale (nullable): the E4M3 copy of m with one scale per row.
 cudaError_t launch_latent_reduce(const __nv_bfloat16* y, const int* inv, const float* w,
-                                 __nv_bfloat16* m, int T, int k, int L, cudaStream_t stream);
+                                 __nv_bfloat16* m, uint8_t* mq, float* m_scale, int T, int k,
+                                 int L, cudaStream_t stream);
 
 }  // namespace moe

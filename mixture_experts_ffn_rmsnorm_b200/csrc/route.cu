@@ -248,18 +248,36 @@ __global__ void __launch_bounds__(256) router_reduce_kernel(
   if (lane < k && unsigned(e) < unsigned(E)) atomicAdd(hist + size_t(t / kBM) * E + e, 1);
 }
 
-// uq[p] = E4M3(u[p] / s_p), s_p = amax_p / 448; amax_p reset to 0 for the
-// next forward.  One block per row.
+// E4M3 copy of a row set: q[p] = E4M3(x[p] / s_p), s_p = amax_p / 448, and
+// amax_p reset to 0 for the next forward.  One block per row; blocks
+// [0, R) take the rows of the first set (routed relu^2(up), width I),
+// blocks [R, R + Rv) those of the second (shared relu^2(up), width S).
 __global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ u,
-                                     unsigned* __restrict__ amax, uint8_t* __restrict__ uq,
-                                     float* __restrict__ scale, int I) {
-  const int p = blockIdx.x;
+                                     unsigned* __restrict__ u_amax, uint8_t* __restrict__ uq,
+                                     float* __restrict__ u_scale, int R, int I,
+                                     const __nv_bfloat16* __restrict__ v,
+                                     unsigned* __restrict__ v_amax, uint8_t* __restrict__ vq,
+                                     float* __restrict__ v_scale, int S) {
+  int p = blockIdx.x;
+  const __nv_bfloat16* x = u;
+  unsigned* amax = u_amax;
+  uint8_t* q = uq;
+  float* scale = u_scale;
+  int W = I;
+  if (p >= R) {
+    p -= R;
+    x = v;
+    amax = v_amax;
+    q = vq;
+    scale = v_scale;
+    W = S;
+  }
   const float m = __uint_as_float(amax[p]);
   const float s = m > 0.f ? m / 448.f : 1.f;
   const float inv = 1.f / s;
-  const uint4* src = reinterpret_cast<const uint4*>(u + size_t(p) * I);
-  uint2* dst = reinterpret_cast<uint2*>(uq + size_t(p) * I);
-  for (int i = threadIdx.x; i < I / 8; i += blockDim.x) {
+  const uint4* src = reinterpret_cast<const uint4*>(x + size_t(p) * W);
+  uint2* dst = reinterpret_cast<uint2*>(q + size_t(p) * W);
+  for (int i = threadIdx.x; i < W / 8; i += blockDim.x) {
     float f[8];
     unpack8(src[i], f);
     dst[i] = make_uint2(e4m3x4(f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv),
@@ -453,18 +471,23 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, const int* _
 }
 
 // LatentMoE: m[t] = bf16(sum_j w[t,j] * y[inv[t*k + j]]) in latent space.
+// With FP8 fc2 weights the block also writes the row's E4M3 copy mq[t] with
+// its scale (max |m[t]| / 448): the block owns the whole row.
 __global__ void latent_reduce_kernel(const __nv_bfloat16* __restrict__ y,
                                      const int* __restrict__ inv, const float* __restrict__ w,
-                                     __nv_bfloat16* __restrict__ m, int k, int L) {
+                                     __nv_bfloat16* __restrict__ m, uint8_t* __restrict__ mq,
+                                     float* __restrict__ m_scale, int k, int L) {
   const int t = blockIdx.x;
   __shared__ int rows[kMaxTopKShared];
   __shared__ float wts[kMaxTopKShared];
+  __shared__ float red[32];
   if (threadIdx.x < k) {
     rows[threadIdx.x] = inv[t * k + threadIdx.x];
     wts[threadIdx.x] = w[t * k + threadIdx.x];
   }
   __syncthreads();
   const int nv = L / 8;
+  float amax = 0.f;
   for (int i = threadIdx.x; i < nv; i += blockDim.x) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, f[8];
     for (int j = 0; j < k; ++j) {
@@ -473,7 +496,29 @@ __global__ void latent_reduce_kernel(const __nv_bfloat16* __restrict__ y,
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] += wj * f[q];
     }
-    reinterpret_cast<uint4*>(m + size_t(t) * L)[i] = pack8(acc);
+    const uint4 packed = pack8(acc);
+    reinterpret_cast<uint4*>(m + size_t(t) * L)[i] = packed;
+    unpack8(packed, f);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(f[q]));
+  }
+  if (!mq) return;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  float a = 0.f;
+  for (int i = 0; i < int(blockDim.x >> 5); ++i) a = fmaxf(a, red[i]);
+  const float scale = a > 0.f ? a / 448.f : 1.f;
+  const float rcp = 1.f / scale;
+  if (threadIdx.x == 0) m_scale[t] = scale;
+  // the E4M3 copy of the bf16 row this thread wrote above
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+    float f[8];
+    unpack8(reinterpret_cast<const uint4*>(m + size_t(t) * L)[i], f);
+    reinterpret_cast<uint2*>(mq + size_t(t) * L)[i] =
+        make_uint2(e4m3x4(f[0] * rcp, f[1] * rcp, f[2] * rcp, f[3] * rcp),
+                   e4m3x4(f[4] * rcp, f[5] * rcp, f[6] * rcp, f[7] * rcp));
   }
 }
 
@@ -516,10 +561,13 @@ cudaError_t launch_router_reduce(const float* part, int ks, int rows_cap, int T,
                             idx, w, hist);
 }
 
-cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* amax, uint8_t* uq,
-                                 float* scale, int R, int I, cudaStream_t stream) {
-  if (R <= 0) return cudaSuccess;
-  quantize_rows_kernel<<<R, 128, 0, stream>>>(u, amax, uq, scale, I);
+cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* u_amax, uint8_t* uq,
+                                 float* u_scale, int R, int I, const __nv_bfloat16* v,
+                                 unsigned* v_amax, uint8_t* vq, float* v_scale, int Rv, int S,
+                                 cudaStream_t stream) {
+  if (R + Rv <= 0) return cudaSuccess;
+  quantize_rows_kernel<<<R + Rv, 128, 0, stream>>>(u, u_amax, uq, u_scale, R, I, v, v_amax, vq,
+                                                   v_scale, S);
   return cudaGetLastError();
 }
 
@@ -555,8 +603,9 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int* inv, const float* 
 }
 
 cudaError_t launch_latent_reduce(const __nv_bfloat16* y, const int* inv, const float* w,
-                                 __nv_bfloat16* m, int T, int k, int L, cudaStream_t stream) {
-  latent_reduce_kernel<<<T, 128, 0, stream>>>(y, inv, w, m, k, L);
+                                 __nv_bfloat16* m, uint8_t* mq, float* m_scale, int T, int k,
+                                 int L, cudaStream_t stream) {
+  latent_reduce_kernel<<<T, 128, 0, stream>>>(y, inv, w, m, mq, m_scale, k, L);
   return cudaGetLastError();
 }
 

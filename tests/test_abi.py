@@ -65,7 +65,8 @@ ALL16 = dict(norm_w=16, gate_w=32, gate_bias=None, up_w=48, down_w=64, up_scale=
                                  dict(num_experts=257, top_k=2), dict(hidden_size=100),
                                  dict(moe_inter=96), dict(shared_inter=0), dict(latent_size=-64),
                                  dict(latent_size=32), dict(max_tokens=0), dict(rms_eps=-1.0),
-                                 dict(expert_wdtype=5),
+                                 dict(expert_wdtype=5), dict(shared_wdtype=3),
+                                 dict(latent_wdtype=-1),
                                  dict(routed_scaling_factor=float("inf"))])
 def test_invalid_configs_rejected_on_host(bad):
     # NemotronMoeLayer `new`: top_k must be in 1..=num_experts and within the
@@ -88,6 +89,16 @@ def test_null_and_misaligned_weights_rejected():
     assert st == 2
     st, _ = _create(_cfg(latent_size=128), moe.MoEWeights(**ALL16))
     assert st == 2
+    # FP8 shared expert / fc1 / fc2 need their row scales too
+    st, _ = _create(_cfg(shared_wdtype=1), moe.MoEWeights(**ALL16))
+    assert st == 2
+    lat = dict(ALL16, fc1_w=112, fc2_w=128)
+    st, _ = _create(_cfg(latent_size=128, latent_wdtype=1), moe.MoEWeights(**lat))
+    assert st == 2
+    # FP8 routed experts are wired for the direct layer only
+    st, _ = _create(_cfg(latent_size=128, expert_wdtype=1),
+                    moe.MoEWeights(**dict(lat, up_scale=144, down_scale=160)))
+    assert st == 1
 
 
 def test_invalid_handle_rejected():

@@ -31,12 +31,9 @@ def test_decode_T1_bytes_match_the_weight_stream():
     closed = weights + tokens
     assert closed == 160_355_328  # 160.4 MB: a 24.5 us roofline at 6.53 TB/s
     model = bench.stage_model(s, T, "decode", U)
-    assert [m[0] for m in model] == ["decode_route", "decode_up_gemm", "decode_down_gemm"]
-    # the model adds the intermediate activations (R x I, T x S) both ways
-    assert _sum(model, 1) == pytest.approx(closed, rel=1e-3)
-    up, down = model[1], model[2]
-    assert up[1] - (U * I * H * 2 + S * H * 2) < 64 * 1024
-    assert down[1] - (U * H * I * 2 + H * S * 2) < 64 * 1024
+    assert [m[0] for m in model] == ["decode_fused"]  # the decode path is one launch
+    assert model[0][1] == closed
+    assert model[0][2] == 2 * T * H * E + 4 * T * k * H * I + 4 * T * H * S
 
 
 @pytest.mark.parametrize("name,T,gflop", [
