@@ -59,8 +59,8 @@ struct FusedDecodeArgs {
 };
 
 // Whether the single-launch decode path covers this configuration (direct
-// layer, BF16 routed and shared experts).
-bool fused_decode_supported(const moe_config& c);
+// layer, BF16 routed and shared experts) on a grid of `grid` CTAs.
+bool fused_decode_supported(const moe_config& c, int grid);
 cudaError_t prepare_fused_decode();
 cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream);
 

@@ -312,7 +312,7 @@ bool build_maps(moe_handle* h) {
   ok &= make_map(&h->tm_sup_w, h->w.shared_up_w, sf8, H, S, H * sb, h->up_bn);
   ok &= make_map(&h->tm_down_w, h->w.down_w, f8, I, E * D, I * eb, h->down_bn);
   ok &= make_map(&h->tm_sdown_w, h->w.shared_down_w, sf8, S, H, S * sb, h->down_bn);
-  if (moe::fused_decode_supported(c))
+  if (moe::fused_decode_supported(c, h->num_sms))
     ok &= make_map(&h->tm_dec_x, h->dec.x16, false, H, uint64_t(h->num_sms) * moe::kDecodeN,
                    H * 2, moe::kDecodeN);
   return ok;
@@ -530,7 +530,7 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
 moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cudaStream_t st,
                           moe::LaunchLog* log) {
   const moe_config& c = h->cfg;
-  if (!moe::fused_decode_supported(c) || T < 1 || T > MOE_DECODE_MAX_TOKENS)
+  if (!moe::fused_decode_supported(c, h->num_sms) || T < 1 || T > MOE_DECODE_MAX_TOKENS)
     return MOE_ERR_INVALID_CONFIG;
   moe::FusedDecodeArgs a;
   a.cfg = &c;
@@ -651,7 +651,7 @@ moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t
   log.begin(s);
   const bool decode = path == MOE_PATH_DECODE ||
                       (path == MOE_PATH_AUTO && num_tokens <= MOE_DECODE_MAX_TOKENS &&
-                       moe::fused_decode_supported(h->cfg));
+                       moe::fused_decode_supported(h->cfg, h->num_sms));
   if (decode) {
     st = enqueue_decode(h, static_cast<bf16*>(hidden), static_cast<bf16*>(residual), num_tokens,
                         s, &log);
