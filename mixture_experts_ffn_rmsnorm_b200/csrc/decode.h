@@ -50,7 +50,7 @@ struct FusedDecodeArgs {
   const moe_weights* w;
   const FusedWorkspace* ws;
   const CUtensorMap *tm_up, *tm_sup, *tm_down, *tm_sdown;  // weights as 128-row A boxes
-  const CUtensorMap* tm_x;                                 // token rows, 16-row B boxes
+  const CUtensorMap* tm_x[4];  // token rows, B boxes of 1, 2, 4, 8 rows (token-count bucket)
   __nv_bfloat16* hidden;
   __nv_bfloat16* residual;
   int T;

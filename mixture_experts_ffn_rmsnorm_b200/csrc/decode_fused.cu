@@ -75,6 +75,7 @@ constexpr int kReduceParts = 8;
 // Named barriers (0 is __syncthreads).
 constexpr int kBarEpi = 1;
 constexpr int kBarRoute = 2;
+constexpr int kBarAll = 3;  // all kThreads threads (the final reduction)
 
 // Synchronisation words of the workspace (FusedWorkspace::sync).
 enum { kRouteArrived = 0, kPartialsDone = 1, kExited = 2 };
@@ -84,7 +85,7 @@ struct FusedParams {
   CUtensorMap tm_sup;    // shared up weights   [S, H]
   CUtensorMap tm_down;   // routed down weights [E*H, I]
   CUtensorMap tm_sdown;  // shared down weights [H, S]
-  CUtensorMap tm_x;      // x16 [grid * 16, H]: 16 rows per CTA   (B, 16-row boxes)
+  CUtensorMap tm_x;      // x16 [grid * 16, H]: 16 rows per CTA   (B, boxes of MAXT rows)
   const bf16* hidden;
   bf16* residual;
   bf16* out;             // = hidden (written at the very end)
@@ -179,6 +180,7 @@ struct Shared {
   int flag;
   int U;                    // routed slots
   float rs[kDecodeMaxT];
+  float4 dry4[1 + kReduceParts];  // the dry reduction pass's staging
   float red[4][kDecodeMaxT * 3];
   int seg_expert[kMaxSlots];            // expert of routed slot s
   float seg_w[kMaxSlots][kDecodeN];     // routing weight of token t in slot s (0 = not routed)
@@ -254,9 +256,13 @@ __device__ __forceinline__ bool step_of(const Units& u, int m, int s, int* kind,
 
 // ---------------------------------------------------------------- routing
 // Routing warps (rt 0..127).  One pass over the tokens, the norm weight and
-// this CTA's gate rows (blockIdx.x and, with E > grid, blockIdx.x + grid):
-// the sums of squares and the dot products G_e . (x_t * w) come out of the
-// same loads.  CTA 0 also writes the normed rows and the residual.
+// this CTA's gate rows (blockIdx.x and, with E > grid, blockIdx.x + grid)
+// gives everything at once: the sums of squares, the dot products
+// G_e . (x_t * w), this CTA's copy of the token rows bf16(x * w) for the up
+// GEMM, and (CTA 0) the residual.  The up GEMM's token operand leaves out
+// the factor r_t = rsqrt(mean x_t^2 + eps), so it needs nothing but the
+// loads; the epilogue applies r_t to accumulator column t instead
+// (W . (x r w) = r (W . (x w))).
 template <int MAXT>
 __device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
   const int H = p.H, T = p.T, E = p.E, G = gridDim.x;
@@ -264,13 +270,12 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
   const int warp = rt >> 5, lane = rt & 31;
   const int e0 = blockIdx.x, e1 = blockIdx.x + G;
   const bool has0 = e0 < E, has1 = e1 < E;
-  // One or two tokens: every chunk's loads in flight first, the token chunks
-  // kept in registers for the normed rows below.  More tokens would spill
-  // those registers: their chunks are loaded one at a time, and again for
-  // the normed rows.
+  bf16* x16 = p.ws.x16 + size_t(blockIdx.x) * kDecodeN * H;
+  // One or two tokens: every chunk's loads in flight at once.  More tokens
+  // would spill those registers: their chunks go one at a time.
   constexpr bool kHold = MAXT <= 2;
   constexpr int kHeld = kHold ? kMaxChunks : 1;
-  uint4 xv[kHeld][MAXT], wv[kHeld];
+  uint4 xv[kHeld][MAXT], wv[kHeld], g0[kHeld], g1[kHeld];
   auto load_chunk = [&](int j, uint4 (&x)[MAXT], uint4& w, uint4& a, uint4& b) {
     const int c = rt + j * kRouteThreads;
     const bool in = c < nv;
@@ -287,8 +292,10 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
   float ss[MAXT], d0[MAXT], d1[MAXT];
 #pragma unroll
   for (int t = 0; t < MAXT; ++t) ss[t] = d0[t] = d1[t] = 0.f;
-  auto accumulate = [&](const uint4 (&x)[MAXT], const uint4& wq, const uint4& aq,
-                        const uint4& bq) {
+  // sums of chunk j, and its token rows bf16(x * w) (and the residual)
+  auto consume = [&](int j, const uint4 (&x)[MAXT], const uint4& wq, const uint4& aq,
+                     const uint4& bq) {
+    const int c = rt + j * kRouteThreads;
     float w[8], a[8], b[8];
     unpack8(wq, w);
     unpack8(aq, a);
@@ -308,20 +315,24 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
         d0[t] += a[q] * f[q];
         d1[t] += b[q] * f[q];
       }
+      if (c < nv && t < T) {
+        reinterpret_cast<uint4*>(x16 + size_t(t) * H)[c] =
+            make_uint4(pack_bf16x2(f[0] * w[0], f[1] * w[1]), pack_bf16x2(f[2] * w[2], f[3] * w[3]),
+                       pack_bf16x2(f[4] * w[4], f[5] * w[5]), pack_bf16x2(f[6] * w[6], f[7] * w[7]));
+        if (blockIdx.x == 0) reinterpret_cast<uint4*>(p.residual + size_t(t) * H)[c] = x[t];
+      }
     }
   };
   if constexpr (kHold) {
-    uint4 g0[kMaxChunks], g1[kMaxChunks];
 #pragma unroll
     for (int j = 0; j < kMaxChunks; ++j) load_chunk(j, xv[j], wv[j], g0[j], g1[j]);
 #pragma unroll
-    for (int j = 0; j < kMaxChunks; ++j) accumulate(xv[j], wv[j], g0[j], g1[j]);
+    for (int j = 0; j < kMaxChunks; ++j) consume(j, xv[j], wv[j], g0[j], g1[j]);
   } else {
 #pragma unroll 1
     for (int j = 0; j < kMaxChunks; ++j) {
-      uint4 g0, g1;
-      load_chunk(j, xv[0], wv[0], g0, g1);
-      accumulate(xv[0], wv[0], g0, g1);
+      load_chunk(j, xv[0], wv[0], g0[0], g1[0]);
+      consume(j, xv[0], wv[0], g0[0], g1[0]);
     }
   }
   if (rt < E) sh.bias[rt] = p.gate_bias ? p.gate_bias[rt] : 0.f;
@@ -336,6 +347,8 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
       sh.red[warp][2 * MAXT + t] = v2;
     }
   }
+  // the token rows: generic writes -> the TMA loads of this CTA's producer
+  fence_proxy_async_global();
   named_barrier(kBarRoute, kRouteThreads);
   // the routing loads have returned (their sums are in shared memory): the
   // weight stream may start.  Routing decides when the routed weights can
@@ -354,56 +367,12 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
     if (has1) p.ws.logits[rt * E + e1] = b * r;
   }
   named_barrier(kBarRoute, kRouteThreads);
-  // this CTA's copy of the normed rows n = x * r * w (bf16), for its own
-  // TMA loads
-  bf16* x16 = p.ws.x16 + size_t(blockIdx.x) * kDecodeN * H;
-#pragma unroll
-  for (int j = 0; j < kMaxChunks; ++j) {
-    const int c = rt + j * kRouteThreads;
-    if (c < nv) {
-      const int hj = kHold ? j : 0;
-      if (!kHold) {
-        wv[0] = __ldg(reinterpret_cast<const uint4*>(p.norm_w) + c);
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t)
-          if (t < T) xv[0][t] = reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c];
-      }
-      float w[8];
-      unpack8(wv[hj], w);
-#pragma unroll
-      for (int t = 0; t < MAXT; ++t) {
-        if (t < T) {
-          float f[8];
-          unpack8(xv[hj][t], f);
-          const float r = sh.rs[t];
-          reinterpret_cast<uint4*>(x16 + size_t(t) * H)[c] =
-              make_uint4(pack_bf16x2(f[0] * r * w[0], f[1] * r * w[1]),
-                         pack_bf16x2(f[2] * r * w[2], f[3] * r * w[3]),
-                         pack_bf16x2(f[4] * r * w[4], f[5] * r * w[5]),
-                         pack_bf16x2(f[6] * r * w[6], f[7] * r * w[7]));
-        }
-      }
-    }
+  // the token rows and their factors r_t are in place; every logit of this
+  // CTA is written (and, CTA 0, the residual)
+  if (rt == 0) {
+    mbar_arrive(&sh.tokens);
+    red_release_add(p.ws.sync + kRouteArrived, 1u);
   }
-  fence_proxy_async_global();
-  named_barrier(kBarRoute, kRouteThreads);
-  if (rt == 0) mbar_arrive(&sh.tokens);
-  if (blockIdx.x == 0) {  // the residual
-#pragma unroll
-    for (int j = 0; j < kMaxChunks; ++j) {
-      const int c = rt + j * kRouteThreads;
-      if (c < nv) {
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t)
-          if (t < T)
-            reinterpret_cast<uint4*>(p.residual + size_t(t) * H)[c] =
-                kHold ? xv[kHold ? j : 0][t]
-                      : reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c];
-      }
-    }
-  }
-  named_barrier(kBarRoute, kRouteThreads);
-  if (rt == 0) red_release_add(p.ws.sync + kRouteArrived, 1u);
 }
 
 // Once every CTA's logits are in: the sigmoid top-k of every token and the
@@ -532,6 +501,82 @@ __device__ __forceinline__ UnitInfo unit_info(const FusedParams& p, const Shared
 // of an expert may have only 64 valid rows).
 __device__ __forceinline__ int down_kk(const UnitInfo& f) { return f.rows - f.row0 >= kBM ? 2 : 1; }
 
+// ------------------------------------------------------------ reduction
+// Output rows [r0, r0 + nr) of T tokens: the partials of CTAs 0..active-1,
+// added in CTA order (deterministic), plus the input row, into out.  Run by
+// `nthreads` threads meeting at barrier `bar`; the partials are staged in
+// shared memory at stage4 (the idle ring).
+//
+// Like route_select it also runs once as a dry pass at the start of the
+// launch (epilogue warps, one source, four rows, a scratch area, no store),
+// so that its instructions are in the cache when the real pass comes last
+// on the critical path.  Not inlined, so that both passes run the same code.
+__device__ __noinline__ void reduce_slice(const FusedParams& p, float4* stage4, int T, int active,
+                                          int r0, int nr, int tid, int nthreads, int bar,
+                                          bool dry) {
+  const int H = p.H;
+  // stage every partial value of the slice, [source CTA][token][row], four
+  // rows per load; each thread has up to kBatch loads in flight before it
+  // stores any
+  constexpr int kBatch = 4;
+  const int nq = nr >> 2;
+  const int per = T * nq;
+  const int count = active * per;
+  for (int i0 = tid; i0 < count; i0 += kBatch * nthreads) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * nthreads;
+      if (i < count) {
+        const int src = i / per, rem = i - src * per;
+        const int t = rem / nq, q = rem - t * nq;
+        v[u] = __ldcg(reinterpret_cast<const float4*>(
+                          p.ws.part + (size_t(src) * kDecodeMaxT + t) * H + r0) + q);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (i0 + u * nthreads < count) stage4[i0 + u * nthreads] = v[u];
+  }
+  named_barrier(bar, nthreads);
+  // each output is summed by kParts threads over fixed, consecutive source
+  // ranges, then the kParts sums in order: a fixed order
+  constexpr int kParts = kReduceParts;
+  float4* sums = stage4 + count;  // [per][kParts]
+  const int span = (active + kParts - 1) / kParts;
+  for (int i = tid; i < per * kParts; i += nthreads) {
+    const int o = i / kParts, part = i - o * kParts;
+    const int s0 = part * span, s1 = min(active, s0 + span);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int src = s0; src < s1; ++src) {
+      const float4 v = stage4[src * per + o];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    sums[i] = acc;
+  }
+  named_barrier(bar, nthreads);
+  for (int o = tid; o < per; o += nthreads) {
+    const int t = o / nq, row = r0 + (o - t * nq) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int part = 0; part < kParts; ++part) {
+      const float4 v = sums[o * kParts + part];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    const size_t at = size_t(t) * H + row;
+    const uint2 hv = *reinterpret_cast<const uint2*>(p.hidden + at);
+    const uint2 ov = make_uint2(pack_bf16x2(lo16(hv.x) + acc.x, hi16(hv.x) + acc.y),
+                                pack_bf16x2(lo16(hv.y) + acc.z, hi16(hv.y) + acc.w));
+    if (!dry) *reinterpret_cast<uint2*>(p.out + at) = ov;
+  }
+}
+
 // ---------------------------------------------------------------- kernel
 template <int MAXT>
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ FusedParams p) {
@@ -644,7 +689,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           }
         }
         uint8_t* sa = tiles + stage * kStageBytes;
-        mbar_arrive_expect_tx(&sh.full[stage], uint32_t(nk * (up ? kABytes + kBBytes : kABytes)));
+        // (a token box holds MAXT rows: the MMA reads all 16 rows of the slot,
+        // but rows past T only reach accumulator columns the epilogue drops)
+        mbar_arrive_expect_tx(&sh.full[stage], uint32_t(nk * (up ? kABytes + MAXT * 128 : kABytes)));
         for (int i = 0; i < nk; ++i) tma_load_2d(sa + i * kABytes, map, &sh.full[stage], ax + i * 64, ay);
         if (up) {
           if (npend) flush(false);
@@ -842,6 +889,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     // the dry routing pass (see route_select), then the real one may start
     route_select(p, sh, tid, abort, kBarEpi, true);
     if (tid == 0) mbar_arrive(&sh.warm);
+    // and the final reduction's (one source, one token, four rows)
+    reduce_slice(p, sh.dry4, 1, 1, 0, 4, tid, kEpiThreads, kBarEpi, true);
+    // the factors r_t of the token rows (published with the rows)
+    if (lane == 0 && !mbar_wait(&sh.tokens, 0, abort)) record_timeout(p.status, abort);
+    __syncwarp();
+    float rsc[kDecodeN];
+#pragma unroll
+    for (int c = 0; c < kDecodeN; ++c) rsc[c] = c < MAXT && c < p.T ? sh.rs[c] : 0.f;
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int rloc = q * 32 + lane;
     const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
@@ -886,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
 #pragma unroll
       for (int c = 0; c < kDecodeN; ++c) {
         const float w = f.shared ? (c < p.T ? 1.f : 0.f) : sh.seg_w[f.slot][c];
-        const float a = __uint_as_float(r[c]);
+        const float a = __uint_as_float(r[c]) * rsc[c];
         v[c] = valid && w != 0.f ? (a > 0.f ? a * a : 0.f) * w : 0.f;
       }
       // buffer b is free once unit n - 2's down MMAs have completed
@@ -955,73 +1010,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   }
   __syncthreads();
   if (!*abort) {
-    const int T = p.T, H = p.H;
     const int active = n_units < G ? n_units : G;
-    const int R0 = reduce_rows(H, G);
+    const int R0 = reduce_rows(p.H, G);
     const int r0 = cta * R0;
-    const int nr = min(H, r0 + R0) - r0;  // a multiple of 4: H is one of 64
-    if (nr > 0) {
-      // stage every partial value of the slice in shared memory (the ring
-      // is idle now), [source CTA][token][row], four rows per load; each
-      // thread has up to four loads in flight before it stores any
-      float4* stage4 = reinterpret_cast<float4*>(tiles);
-      const int nq = nr >> 2;
-      const int per = T * nq;
-      const int count = active * per;
-      for (int i0 = threadIdx.x; i0 < count; i0 += 4 * kThreads) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = i0 + u * kThreads;
-          if (i < count) {
-            const int src = i / per, rem = i - src * per;
-            const int t = rem / nq, q = rem - t * nq;
-            v[u] = __ldcg(reinterpret_cast<const float4*>(
-                              p.ws.part + (size_t(src) * kDecodeMaxT + t) * H + r0) + q);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (i0 + u * kThreads < count) stage4[i0 + u * kThreads] = v[u];
-      }
-      __syncthreads();
-      // each output is summed by kParts threads over fixed, consecutive
-      // source ranges, then the kParts sums in order: a fixed order
-      constexpr int kParts = kReduceParts;
-      float4* sums = stage4 + count;  // [per][kParts]
-      const int span = (active + kParts - 1) / kParts;
-      for (int i = threadIdx.x; i < per * kParts; i += kThreads) {
-        const int o = i / kParts, part = i - o * kParts;
-        const int s0 = part * span, s1 = min(active, s0 + span);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = s0; src < s1; ++src) {
-          const float4 v = stage4[src * per + o];
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
-        }
-        sums[i] = acc;
-      }
-      __syncthreads();
-      for (int o = threadIdx.x; o < per; o += kThreads) {
-        const int t = o / nq, row = r0 + (o - t * nq) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int part = 0; part < kParts; ++part) {
-          const float4 v = sums[o * kParts + part];
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
-        }
-        const size_t at = size_t(t) * H + row;
-        const uint2 hv = *reinterpret_cast<const uint2*>(p.hidden + at);
-        *reinterpret_cast<uint2*>(p.out + at) =
-            make_uint2(pack_bf16x2(lo16(hv.x) + acc.x, hi16(hv.x) + acc.y),
-                       pack_bf16x2(lo16(hv.y) + acc.z, hi16(hv.y) + acc.w));
-      }
-    }
+    const int nr = min(p.H, r0 + R0) - r0;  // a multiple of 4: H is one of 64
+    if (nr > 0)
+      reduce_slice(p, reinterpret_cast<float4*>(tiles), p.T, active, r0, nr, threadIdx.x,
+                   kThreads, kBarAll, false);
   }
   if (threadIdx.x == 0) {
     // the last CTA out resets the launch's synchronisation words: every
@@ -1077,7 +1072,8 @@ cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   p.tm_sup = *a.tm_sup;
   p.tm_down = *a.tm_down;
   p.tm_sdown = *a.tm_sdown;
-  p.tm_x = *a.tm_x;
+  const int bucket = a.T <= 1 ? 0 : a.T <= 2 ? 1 : a.T <= 4 ? 2 : 3;
+  p.tm_x = *a.tm_x[bucket];
   p.hidden = a.hidden;
   p.residual = a.residual;
   p.out = a.hidden;

@@ -138,7 +138,7 @@ struct moe_handle {
   CUtensorMap tm_up_w, tm_sup_w, tm_down_w, tm_sdown_w;
   int up_bn, down_bn;
   CUtensorMap tm_fc2_a, tm_fc2_b;
-  CUtensorMap tm_dec_x;  // decode token rows, one 16-row block per CTA (16-row boxes)
+  CUtensorMap tm_dec_x[4];  // decode token rows, one 16-row block per CTA; boxes of 1, 2, 4, 8 rows
 };
 
 namespace {
@@ -313,8 +313,9 @@ bool build_maps(moe_handle* h) {
   ok &= make_map(&h->tm_down_w, h->w.down_w, f8, I, E * D, I * eb, h->down_bn);
   ok &= make_map(&h->tm_sdown_w, h->w.shared_down_w, sf8, S, H, S * sb, h->down_bn);
   if (moe::fused_decode_supported(c, h->num_sms))
-    ok &= make_map(&h->tm_dec_x, h->dec.x16, false, H, uint64_t(h->num_sms) * moe::kDecodeN,
-                   H * 2, moe::kDecodeN);
+    for (int b = 0; b < 4; ++b)
+      ok &= make_map(&h->tm_dec_x[b], h->dec.x16, false, H, uint64_t(h->num_sms) * moe::kDecodeN,
+                     H * 2, 1u << b);
   return ok;
 }
 
@@ -540,7 +541,7 @@ moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cu
   a.tm_sup = &h->tm_sup_b;    // shared up weights [S, H]
   a.tm_down = &h->tm_down_b;  // routed down weights [E*H, I]
   a.tm_sdown = &h->tm_sdown_b;
-  a.tm_x = &h->tm_dec_x;
+  for (int b = 0; b < 4; ++b) a.tm_x[b] = &h->tm_dec_x[b];
   a.hidden = hidden;
   a.residual = residual;
   a.T = T;
