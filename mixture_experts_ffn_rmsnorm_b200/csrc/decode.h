@@ -21,16 +21,18 @@ constexpr int kDecodeN = 16;  // token columns of a decode tile (UMMA N)
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 // Workspace of the single-launch decode path (decode_fused.cu).  The
-// synchronisation words start at zero (the workspace is cleared at
-// creation) and every launch leaves them at zero: the last CTA to exit
-// resets them.
+// synchronisation words, the accumulator and the marks start at zero (the
+// workspace is cleared at creation) and every launch leaves them at zero:
+// each CTA clears the accumulator rows it finishes, and the last CTA to exit
+// resets the synchronisation words.
 struct FusedWorkspace {
   __nv_bfloat16* x16;      // [CTAs, 16, H] each CTA's copy of bf16(n) of the tokens (rows >= T unused)
   float* logits;           // [8, E]
   int* idx;                // [8, k] routing of the pass (for moe_copy_routing)
   float* w;                // [8, k]
-  float* part;             // [CTAs, 8, H] each CTA's partial output (token-major)
-  unsigned* sync;          // [4] logit arrivals, partial outputs stored, exited CTAs
+  long long* acc;          // [8, H] fixed-point sum of the CTAs' partial outputs (token-major)
+  uint8_t* bad;            // [8, H] 1 where a partial was not finite or out of range
+  unsigned* sync;          // [4] logit arrivals, partial outputs added, exited CTAs
 };
 
 // ctas: grid of the decode launch (one CTA per SM).
@@ -41,7 +43,8 @@ void carve_fused(FusedWorkspace* d, const moe_config& c, int ctas, Take take) {
   d->logits = reinterpret_cast<float*>(take(kDecodeMaxT * E * 4));
   d->idx = reinterpret_cast<int*>(take(kDecodeMaxT * k * 4));
   d->w = reinterpret_cast<float*>(take(kDecodeMaxT * k * 4));
-  d->part = reinterpret_cast<float*>(take(size_t(ctas) * kDecodeMaxT * H * 4));
+  d->acc = reinterpret_cast<long long*>(take(kDecodeMaxT * H * 8));
+  d->bad = reinterpret_cast<uint8_t*>(take(kDecodeMaxT * H));
   d->sync = reinterpret_cast<unsigned*>(take(4 * 4));
 }
 

@@ -67,15 +67,23 @@ constexpr int kTmemCols = 512;              // 2 x 16 (up) + ceil(H / 128) x 16 
 constexpr int kMaxRowTiles = kTmemCols / kDecodeN - 2;
 constexpr int kSmem = kStages * kStageBytes + 2 * kUBytes + 1024 + 1024;
 
-// Output rows of the final reduction per CTA: ceil(H / grid), rounded up to
-// a multiple of 4 (float4 loads of the partials).
+// Output rows that each CTA finishes: ceil(H / grid), rounded up to a
+// multiple of 4 (vector loads and stores).
 __host__ __device__ constexpr int reduce_rows(int H, int G) { return ((H + G - 1) / G + 3) & ~3; }
-constexpr int kReduceParts = 8;
+
+// The CTAs' partial outputs add up in a fixed-point accumulator: partial x
+// is added as round(x * 2^24) to an int64, so the sum is exact and does not
+// depend on the order in which the CTAs finish (every replay gives the same
+// bits).  The rounding costs at most 2^-25 per partial, far below the bf16
+// rounding of the result.  A partial that is NaN, infinite or larger than
+// 2^31 in magnitude (where 148 of them could overflow the int64) marks its
+// output element, which then comes out NaN.
+constexpr float kFixScale = 16777216.0f;   // 2^24
+constexpr float kFixLimit = 2147483648.0f;  // 2^31
 
 // Named barriers (0 is __syncthreads).
 constexpr int kBarEpi = 1;
 constexpr int kBarRoute = 2;
-constexpr int kBarAll = 3;  // all kThreads threads (the final reduction)
 
 // Synchronisation words of the workspace (FusedWorkspace::sync).
 enum { kRouteArrived = 0, kPartialsDone = 1, kExited = 2 };
@@ -180,7 +188,6 @@ struct Shared {
   int flag;
   int U;                    // routed slots
   float rs[kDecodeMaxT];
-  float4 dry4[1 + kReduceParts];  // the dry reduction pass's staging
   float red[4][kDecodeMaxT * 3];
   int seg_expert[kMaxSlots];            // expert of routed slot s
   float seg_w[kMaxSlots][kDecodeN];     // routing weight of token t in slot s (0 = not routed)
@@ -502,78 +509,49 @@ __device__ __forceinline__ UnitInfo unit_info(const FusedParams& p, const Shared
 __device__ __forceinline__ int down_kk(const UnitInfo& f) { return f.rows - f.row0 >= kBM ? 2 : 1; }
 
 // ------------------------------------------------------------ reduction
-// Output rows [r0, r0 + nr) of T tokens: the partials of CTAs 0..active-1,
-// added in CTA order (deterministic), plus the input row, into out.  Run by
-// `nthreads` threads meeting at barrier `bar`; the partials are staged in
-// shared memory at stage4 (the idle ring).
+// Adds this CTA's partial value v of output element `at` (token-major
+// [T, H]) into the fixed-point accumulator.
+__device__ __forceinline__ void add_partial(const FusedWorkspace& ws, size_t at, float v) {
+  if (fabsf(v) <= kFixLimit)  // (false for NaN)
+    atomicAdd(reinterpret_cast<unsigned long long*>(ws.acc + at),
+              static_cast<unsigned long long>(__float2ll_rn(v * kFixScale)));
+  else
+    ws.bad[at] = 1;
+}
+
+// Output rows [r0, r0 + nr) of T tokens, once every CTA has added its
+// partial: the accumulated sum plus the input row, rounded once to bf16,
+// into out; the accumulator and the marks of these elements are left at
+// zero for the next launch.  Four rows per thread and step.
 //
 // Like route_select it also runs once as a dry pass at the start of the
-// launch (epilogue warps, one source, four rows, a scratch area, no store),
-// so that its instructions are in the cache when the real pass comes last
-// on the critical path.  Not inlined, so that both passes run the same code.
-__device__ __noinline__ void reduce_slice(const FusedParams& p, float4* stage4, int T, int active,
-                                          int r0, int nr, int tid, int nthreads, int bar,
-                                          bool dry) {
+// launch (epilogue warps, one token, four rows, no store), so that its
+// instructions are in the cache when the real pass comes last on the
+// critical path.  Not inlined, so that both passes run the same code.
+__device__ __noinline__ void finish_slice(const FusedParams& p, int T, int r0, int nr, int tid,
+                                          int nthreads, bool dry) {
   const int H = p.H;
-  // stage every partial value of the slice, [source CTA][token][row], four
-  // rows per load; each thread has up to kBatch loads in flight before it
-  // stores any
-  constexpr int kBatch = 4;
   const int nq = nr >> 2;
-  const int per = T * nq;
-  const int count = active * per;
-  for (int i0 = tid; i0 < count; i0 += kBatch * nthreads) {
-    float4 v[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int i = i0 + u * nthreads;
-      if (i < count) {
-        const int src = i / per, rem = i - src * per;
-        const int t = rem / nq, q = rem - t * nq;
-        v[u] = __ldcg(reinterpret_cast<const float4*>(
-                          p.ws.part + (size_t(src) * kDecodeMaxT + t) * H + r0) + q);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-      if (i0 + u * nthreads < count) stage4[i0 + u * nthreads] = v[u];
-  }
-  named_barrier(bar, nthreads);
-  // each output is summed by kParts threads over fixed, consecutive source
-  // ranges, then the kParts sums in order: a fixed order
-  constexpr int kParts = kReduceParts;
-  float4* sums = stage4 + count;  // [per][kParts]
-  const int span = (active + kParts - 1) / kParts;
-  for (int i = tid; i < per * kParts; i += nthreads) {
-    const int o = i / kParts, part = i - o * kParts;
-    const int s0 = part * span, s1 = min(active, s0 + span);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int src = s0; src < s1; ++src) {
-      const float4 v = stage4[src * per + o];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    sums[i] = acc;
-  }
-  named_barrier(bar, nthreads);
-  for (int o = tid; o < per; o += nthreads) {
-    const int t = o / nq, row = r0 + (o - t * nq) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int part = 0; part < kParts; ++part) {
-      const float4 v = sums[o * kParts + part];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    const size_t at = size_t(t) * H + row;
+  for (int i = tid; i < T * nq; i += nthreads) {
+    const int t = i / nq;
+    const size_t at = size_t(t) * H + r0 + (i - t * nq) * 4;
+    const longlong2 q0 = __ldcg(reinterpret_cast<const longlong2*>(p.ws.acc + at));
+    const longlong2 q1 = __ldcg(reinterpret_cast<const longlong2*>(p.ws.acc + at) + 1);
+    const unsigned bad = __ldcg(reinterpret_cast<const unsigned*>(p.ws.bad + at));
     const uint2 hv = *reinterpret_cast<const uint2*>(p.hidden + at);
-    const uint2 ov = make_uint2(pack_bf16x2(lo16(hv.x) + acc.x, hi16(hv.x) + acc.y),
-                                pack_bf16x2(lo16(hv.y) + acc.z, hi16(hv.y) + acc.w));
-    if (!dry) *reinterpret_cast<uint2*>(p.out + at) = ov;
+    const float m[4] = {float(q0.x) * (1.0f / kFixScale), float(q0.y) * (1.0f / kFixScale),
+                        float(q1.x) * (1.0f / kFixScale), float(q1.y) * (1.0f / kFixScale)};
+    const float x[4] = {lo16(hv.x), hi16(hv.x), lo16(hv.y), hi16(hv.y)};
+    float o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = (bad >> (8 * j)) & 0xffu ? __int_as_float(0x7fc00000) : x[j] + m[j];
+    if (!dry) {
+      *reinterpret_cast<uint2*>(p.out + at) =
+          make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+      reinterpret_cast<longlong2*>(p.ws.acc + at)[0] = make_longlong2(0, 0);
+      reinterpret_cast<longlong2*>(p.ws.acc + at)[1] = make_longlong2(0, 0);
+      if (bad) *reinterpret_cast<unsigned*>(p.ws.bad + at) = 0u;
+    }
   }
 }
 
@@ -662,6 +640,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // the weights are read once per launch: evict them first, keeping the
+      // token rows, logits and the partial outputs in L2
+      const uint64_t stream_policy = l2_policy_evict_first();
       // the routing warps' loads go out first (the routing decides when the
       // routed weights can stream)
       if (!mbar_wait(&sh.loads_out, 0, abort)) {
@@ -692,7 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         // (a token box holds MAXT rows: the MMA reads all 16 rows of the slot,
         // but rows past T only reach accumulator columns the epilogue drops)
         mbar_arrive_expect_tx(&sh.full[stage], uint32_t(nk * (up ? kABytes + MAXT * 128 : kABytes)));
-        for (int i = 0; i < nk; ++i) tma_load_2d(sa + i * kABytes, map, &sh.full[stage], ax + i * 64, ay);
+        for (int i = 0; i < nk; ++i)
+          tma_load_2d_hint(sa + i * kABytes, map, &sh.full[stage], ax + i * 64, ay, stream_policy);
         if (up) {
           if (npend) flush(false);
           for (int i = 0; i < nk; ++i) {
@@ -890,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     route_select(p, sh, tid, abort, kBarEpi, true);
     if (tid == 0) mbar_arrive(&sh.warm);
     // and the final reduction's (one source, one token, four rows)
-    reduce_slice(p, sh.dry4, 1, 1, 0, 4, tid, kEpiThreads, kBarEpi, true);
+    finish_slice(p, 1, 0, 4, tid, kEpiThreads, true);
     // the factors r_t of the token rows (published with the rows)
     if (lane == 0 && !mbar_wait(&sh.tokens, 0, abort)) record_timeout(p.status, abort);
     __syncwarp();
@@ -959,13 +941,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       named_barrier(kBarEpi, kEpiThreads);
       if (tid == 0) mbar_arrive(&sh.ufull[b]);
     }
-    // this CTA's partial output: the H x 16 down accumulator, columns < MAXT
+    // this CTA's partial output (the H x 16 down accumulator, columns < T)
+    // into the launch's fixed-point sum
     if (ok && m > 0) {
       if (lane == 0 && !mbar_wait(&sh.down_done, 0, abort)) record_timeout(p.status, abort);
       __syncwarp();
       if (!epi_stop(sh, tid)) {
         tc_fence_after();
-        float* part = p.ws.part + size_t(cta) * kDecodeMaxT * p.H;
         for (int rt = 0; rt < nH; ++rt) {
           uint32_t r[16];
           tmem_ld_32x32b_x16(lane_base + uint32_t((2 + rt) * kDecodeN), r);
@@ -973,7 +955,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           const int row = rt * kBM + rloc;
           if (row < p.H) {
 #pragma unroll
-            for (int c = 0; c < MAXT; ++c) part[size_t(c) * p.H + row] = __uint_as_float(r[c]);
+            for (int c = 0; c < MAXT; ++c)
+              if (c < p.T) add_partial(p.ws, size_t(c) * p.H + row, __uint_as_float(r[c]));
           }
         }
         tc_fence_before();
@@ -996,11 +979,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
-  // Rows [r0, r0 + nr) of the output: the partials of every CTA that had
-  // units, added in CTA order, plus the input row.  Once every CTA's logits
-  // are in, no CTA reads hidden any more, so the rows can be overwritten.
-  // (every thread takes the unit count from the slot table: only some
-  // roles have updated their own copy of it)
+  // Rows [r0, r0 + nr) of the output, once every CTA that had units has
+  // added its partial and every CTA's logits are in (after that no CTA reads
+  // hidden any more, so the rows can be overwritten).  (Thread 0 takes the
+  // unit count from the slot table: only some roles have updated their own
+  // copy of it.)
   const int n_units = un.nS + sh.U * un.nI;
   if (threadIdx.x == 0 && !*abort) {
     const unsigned active = unsigned(n_units < G ? n_units : G);
@@ -1010,13 +993,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   }
   __syncthreads();
   if (!*abort) {
-    const int active = n_units < G ? n_units : G;
     const int R0 = reduce_rows(p.H, G);
     const int r0 = cta * R0;
     const int nr = min(p.H, r0 + R0) - r0;  // a multiple of 4: H is one of 64
-    if (nr > 0)
-      reduce_slice(p, reinterpret_cast<float4*>(tiles), p.T, active, r0, nr, threadIdx.x,
-                   kThreads, kBarAll, false);
+    if (nr > 0) finish_slice(p, p.T, r0, nr, threadIdx.x, kThreads, false);
   }
   if (threadIdx.x == 0) {
     // the last CTA out resets the launch's synchronisation words: every
@@ -1035,16 +1015,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
 
 bool fused_decode_supported(const moe_config& c, int grid) {
   // the routing warps hold a token row in kMaxChunks 8-element chunks each;
-  // the H x 16 down accumulator fits next to the two up accumulators in TMEM;
-  // the final reduction stages its slice of every CTA's partials (and the
-  // kReduceParts sums) in the idle ring
-  const size_t staged = size_t(grid + kReduceParts) * kDecodeMaxT *
-                        size_t(reduce_rows(c.hidden_size, grid)) * sizeof(float);
+  // the H x 16 down accumulator fits next to the two up accumulators in TMEM
   return grid > 0 && c.latent_size == 0 && c.expert_wdtype == MOE_WEIGHTS_BF16 &&
          c.shared_wdtype == MOE_WEIGHTS_BF16 &&
          c.hidden_size <= kMaxChunks * kRouteThreads * 8 &&
-         (c.hidden_size + kBM - 1) / kBM <= kMaxRowTiles &&
-         staged <= size_t(kStages) * kStageBytes;
+         (c.hidden_size + kBM - 1) / kBM <= kMaxRowTiles;
 }
 
 cudaError_t prepare_fused_decode() {

@@ -6,12 +6,9 @@
 // tiles in the same launch (the always-on shared expert, nemotron_moe.rs
 // `prefill`, or LatentMoE fc1 / fc2), and the router GEMM with the sigmoid
 // top-k routing fused into its epilogue (or, with K split over idle SMs,
-// storing fp32 partial logits for the reduction kernel).  The decode launches
-// (BN = 16: weights as the 128-row operand, tokens as N) use the same kernel
-// with a stream-K schedule; the down launch accumulates all segments of a
-// 128-row output block over their concatenated K.  The grouped up and down
-// launches take their tiles dynamically from a device counter; the router
-// and fc2 launches walk a static round-robin.
+// storing fp32 partial logits for the reduction kernel).  The grouped up and
+// down launches take their tiles dynamically from a device counter; the
+// router and fc2 launches walk a static round-robin.
 //
 // Structure (one CTA per SM, persistent over its tiles):
 //   warp 0   one lane issues TMA loads of A (128 x 128 B) and B (BN x 128 B)
@@ -41,9 +38,9 @@ struct Traits {
   static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kKSteps = 4;                 // 4 x 32 bytes of K per stage
-  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr int kTmemCols = 2 * BN;
   static constexpr int kSmem = STAGES * kStageBytes + 1024 + 512;
-  static_assert(kTmemCols == 32 || kTmemCols == 256 || kTmemCols == 512,
+  static_assert(kTmemCols == 256 || kTmemCols == 512,
                 "TMEM allocation must be a power of two >= 32");
 };
 
@@ -51,110 +48,24 @@ __device__ __forceinline__ int stage_k(const GemmClass& C) { return C.fp8 ? 128 
 
 struct Tile {
   int c;        // class
-  int e;        // group (expert) index; decode: segment
-  int row0;     // first A row; decode: first output row inside the segment
+  int e;        // group (expert) index
+  int row0;     // first A row
   int row_end;  // first row not stored
   int n0;       // first output column
   int brow;     // first B row
   int arow;     // first A row to load
-  int split;    // K split index (dense classes); decode: partial slot of the piece
+  int split;    // K split index (dense classes)
   int k0, k1;   // K-block range [k0, k1); k1 < 0 = through the end
-  int tile;     // decode: index in the tile list
-  int npieces;  // decode: pieces the tile is cut into
 };
 
-// Stream-K schedule of a decode launch (see DecodeEpilogue): tiles 0..n1-1
-// have kb1 k-blocks, the rest kb0; CTA c owns global k-blocks
-// [c * P, (c + 1) * P).
-// In the concatenated mode (down launch) every tile has kb0 = kbs + (segments
-// - 1) * kbi k-blocks: the shared expert's kbs, then kbi per routed slot.
-struct DecSched {
-  int n1, kb1, kb0, ntiles, total, P;
-  int kbs, kbi;  // concatenated mode: k-blocks of the shared / a routed segment
-  __device__ __forceinline__ int start(int t) const {
-    return t < n1 ? t * kb1 : n1 * kb1 + (t - n1) * kb0;
-  }
-  __device__ __forceinline__ int len(int t) const { return t < n1 ? kb1 : kb0; }
-  __device__ __forceinline__ int tile_of(int g) const {
-    const int a = n1 * kb1;
-    return g < a ? g / kb1 : n1 + (g - a) / kb0;
-  }
-  __device__ __forceinline__ int npieces(int t) const {
-    const int a = start(t);
-    return (a + len(t) - 1) / P - a / P + 1;
-  }
-};
-
-// count = *dec_count: tiles in the list, or segments in the concatenated mode.
-__device__ __forceinline__ DecSched dec_sched(const GemmParams& p, int count) {
-  DecSched s;
-  s.kb1 = (p.cls[1].K + 63) / 64;
-  s.kb0 = (p.cls[0].K + 63) / 64;
-  s.kbs = s.kb1;
-  s.kbi = s.kb0;
-  if (p.dec_concat) {
-    s.n1 = 0;
-    s.ntiles = (p.dec.M[0] + kBM - 1) / kBM;
-    s.kb0 = s.kbs + (count - 1) * s.kbi;
-  } else {
-    s.ntiles = count;
-    s.n1 = min(p.dec.n_first, count);
-  }
-  s.total = s.n1 * s.kb1 + (s.ntiles - s.n1) * s.kb0;
-  s.P = max((s.total + int(gridDim.x) - 1) / int(gridDim.x), kDecMinPiece);
-  // With no more tiles than CTAs and tiles of one length, every CTA takes
-  // at most one whole tile: no cut tiles, no partial sums.
-  if (!p.dec_concat && s.ntiles <= int(gridDim.x) && (s.n1 == 0 || s.kb0 == s.kb1))
-    s.P = max(s.P, s.n1 > 0 ? s.kb1 : s.kb0);
-  return s;
-}
-
-// The i-th piece of this CTA's range; false when the range has fewer.
-__device__ __forceinline__ bool dec_piece(const GemmParams& p, const DecSched& s, int i,
-                                          Tile* t) {
-  int g = int(blockIdx.x) * s.P;
-  const int end = min(s.total, g + s.P);
-  for (int j = 0;; ++j) {
-    if (g >= end) return false;
-    const int tile = s.tile_of(g);
-    const int a = s.start(tile), b = a + s.len(tile);
-    if (j == i) {
-      if (p.dec_concat) {  // A/B rows are chosen per k-block by the producer
-        t->c = 1;
-        t->e = 0;
-        t->row0 = tile * kBM;
-        t->row_end = p.dec.M[0];
-        t->brow = 0;
-        t->arow = tile * kBM;
-      } else {
-        const DecodeTile d = p.dec_tiles[tile];
-        t->c = d.cls;
-        t->e = d.seg;
-        t->row0 = d.m0;
-        t->row_end = p.dec.M[d.cls];
-        t->brow = d.brow;
-        t->arow = d.arow;
-      }
-      t->n0 = 0;
-      t->k0 = g - a;
-      t->k1 = min(end, b) - a;
-      t->tile = tile;
-      t->npieces = s.npieces(tile);
-      t->split = tile + int(blockIdx.x);
-      return true;
-    }
-    g = min(end, b);
-  }
-}
-
+// Tile number w of the launch: class 0 (routed groups through the m-tile
+// table, or a dense class with its K splits) for w < W0, then class 1.
 template <int BN>
-__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w, int W0) {
+__device__ __forceinline__ Tile tile_at(const GemmParams& p, int w, int W0) {
   Tile t;
   t.split = 0;
   t.k0 = 0;
   t.k1 = -1;
-  t.tile = w;
-  t.npieces = 1;
   if (w < W0) {
     const int ks = p.cls[0].ksplit > 1 ? p.cls[0].ksplit : 1;
     const int nt = p.cls[0].ntiles * ks;
@@ -215,15 +126,13 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
-// The it-th work item of this CTA: a stream-K piece in decode launches,
-// else tile blockIdx.x + it * gridDim.x.
+// The it-th tile of this CTA in the static schedule: tile blockIdx.x +
+// it * gridDim.x.
 template <int BN>
-__device__ __forceinline__ bool work_item(const GemmParams& p, const DecSched& ds, int W, int W0,
-                                          int it, Tile* t) {
-  if (p.dec_count) return dec_piece(p, ds, it, t);
+__device__ __forceinline__ bool work_item(const GemmParams& p, int W, int W0, int it, Tile* t) {
   const int w = int(blockIdx.x) + it * int(gridDim.x);
   if (w >= W) return false;
-  *t = decode_tile<BN>(p, w, W0);
+  *t = tile_at<BN>(p, w, W0);
   return true;
 }
 
@@ -309,127 +218,6 @@ __device__ __forceinline__ void router_epilogue(const GemmParams& p, const GemmC
     for (int e = ep; e < E; e += 4 * 32) p.expert_hist[size_t(mt) * E + e] = s_hist[e];
 }
 
-// Shared-memory copy of the segment -> expert table (concatenated mode).
-__device__ __forceinline__ int* dec_seg_cache() {
-  __shared__ int s[kDecodeMaxSegs];
-  return s;
-}
-
-// Decode epilogues (BN = 16: 128 weight rows x 16 token columns).
-
-// Up output of one row i of a tile: w_t * relu^2 for a routed slot's tokens
-// (0 where a token is not routed to it), relu^2 for the shared expert.
-__device__ __forceinline__ void dec_up_store(const DecodeEpilogue& d, const Tile& t, int i,
-                                             const float (&a)[16]) {
-  const int M = d.M[t.c];
-  if (i >= M) return;
-  if (t.c == 0) {
-    const float* w = d.seg_w + t.e * 16;
-    __nv_bfloat16* o = d.out_up[0] + size_t(t.e) * 16 * M + i;
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const float wt = w[c];
-      const float v = wt != 0.f ? (a[c] > 0.f ? a[c] * a[c] : 0.f) * wt : 0.f;
-      o[size_t(c) * M] = __float2bfloat16_rn(v);
-    }
-  } else {
-    __nv_bfloat16* o = d.out_up[1] + i;
-#pragma unroll
-    for (int c = 0; c < 16; ++c)
-      if (c < d.T) o[size_t(c) * M] = __float2bfloat16_rn(a[c] > 0.f ? a[c] * a[c] : 0.f);
-  }
-}
-
-__device__ __forceinline__ void store_partial(float* slot_base, int rloc, const uint32_t (&r)[16]) {
-  float4* o = reinterpret_cast<float4*>(slot_base + size_t(rloc) * 16);
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    o[c] = make_float4(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1]),
-                       __uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3]));
-}
-
-// acc[c] += slot rows, for slots [s0, s0 + n) in order (columns c < 8 hold
-// the tokens; T <= 8).
-__device__ __forceinline__ void add_slots(float (&acc)[8], const float* part, int s0, int n,
-                                          int rloc) {
-#pragma unroll 4
-  for (int s = 0; s < n; ++s) {
-    const float4* src =
-        reinterpret_cast<const float4*>(part + (size_t(s0 + s) * kBM + rloc) * 16);
-    const float4 a = __ldcg(src), b = __ldcg(src + 1);
-    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-  }
-}
-
-// A piece that covers its whole up tile stores directly; otherwise every
-// piece stores its partial and the last of the tile's pieces to finish sums
-// them in k order and stores.  Down: every piece stores its partial; the
-// last piece of a 128-row output tile to finish sums the tile's pieces in k
-// order (the shared expert's k-blocks, then each routed slot's), adds the
-// residual and writes hidden.
-__device__ __forceinline__ void decode_epilogue(const GemmParams& p, const DecSched& ds,
-                                                const Tile& t, uint32_t tb, int rloc) {
-  __shared__ int last_flag;
-  const DecodeEpilogue& d = p.dec;
-  const GemmClass& C = p.cls[t.c];
-  uint32_t r[16];
-  tmem_ld_32x32b_x16(tb, r);
-  tmem_ld_wait();
-  const int i = t.row0 + rloc;  // output row inside the segment's matrix
-  if (C.epi == EPI_DEC_UP) {
-    if (t.npieces == 1) {
-      float a[16];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) a[c] = __uint_as_float(r[c]);
-      dec_up_store(d, t, i, a);
-      return;
-    }
-    store_partial(d.up_part + size_t(t.split) * kBM * 16, rloc, r);
-    __threadfence();
-    named_barrier(1, 4 * 32);
-    if (threadIdx.x == 2 * 32)
-      last_flag = atomicAdd(d.up_counter + t.tile, 1u) == unsigned(t.npieces - 1);
-    named_barrier(1, 4 * 32);
-    if (!last_flag) return;
-    __threadfence();
-    const int s0 = t.tile + ds.start(t.tile) / ds.P;  // slot of the tile's first piece
-    float acc[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-    add_slots(acc, d.up_part, s0, t.npieces, rloc);
-    float a[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) a[c] = c < 8 ? acc[c] : 0.f;
-    dec_up_store(d, t, i, a);
-    if (threadIdx.x == 2 * 32) d.up_counter[t.tile] = 0u;
-    return;
-  }
-  // down (concatenated mode: a tile is one 128-row block of the output and
-  // its pieces cover every segment's k-blocks)
-  store_partial(d.partial + size_t(t.split) * kBM * 16, rloc, r);
-  __threadfence();
-  named_barrier(1, 4 * 32);
-  if (threadIdx.x == 2 * 32)
-    last_flag = atomicAdd(d.mt_counter + t.tile, 1u) == unsigned(t.npieces - 1);
-  named_barrier(1, 4 * 32);
-  if (!last_flag) return;
-  __threadfence();
-  float acc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-  add_slots(acc, d.partial, t.tile + ds.start(t.tile) / ds.P, t.npieces, rloc);
-  const int M = d.M[t.c];
-  if (i < M) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      if (c < d.T)
-        d.hidden[size_t(c) * M + i] =
-            __float2bfloat16_rn(__bfloat162float(d.residual[size_t(c) * M + i]) + acc[c]);
-  }
-  if (threadIdx.x == 2 * 32) d.mt_counter[t.tile] = 0u;
-}
-
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
@@ -486,68 +274,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   // Everything above overlaps the previous kernel when launched with PDL.
   // Dependents may start once every CTA is past its wait, i.e. once this
-  // launch's own inputs are complete.  In the concatenated decode mode the
-  // producer warp reads the routing tables and its lane 0 issues the first
-  // weight loads before waiting.
-  const bool early_a = BN == 16 && p.dec_concat && warp == 0;
-  if (!early_a) {
-    if (threadIdx.x == 32 && (p.l2_prefetch[0] || p.l2_prefetch[1])) {
-      // a share of weights that do not depend on the previous launch
-      for (int r = 0; r < 2; ++r) {
-        const size_t n = p.l2_prefetch_bytes[r];
-        const size_t per = (n / gridDim.x + 4095) / 4096 * 4096;
-        const size_t b0 = size_t(blockIdx.x) * per;
-        const size_t b1 = min(n, b0 + per);
-        for (size_t b = b0; b < b1; b += 65536)
-          l2_prefetch_bulk(static_cast<const char*>(p.l2_prefetch[r]) + b,
-                           uint32_t(min(size_t(65536), b1 - b)));
-      }
-    }
-    pdl_wait();
-    pdl_trigger();
-  }
+  // launch's own inputs are complete.
+  pdl_wait();
+  pdl_trigger();
 
-  int W0 = 0, W = 0;
-  DecSched ds = {};
-  if (p.dec_count) {
-    ds = dec_sched(p, *p.dec_count);
-  } else {
-    const int m0 = p.n_mtiles ? *p.n_mtiles : p.cls[0].mtiles;
-    W0 = m0 * p.cls[0].ntiles * (p.cls[0].ksplit > 1 ? p.cls[0].ksplit : 1);
-    const int W1 = p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0;
-    W = W0 + W1;
-  }
-  const bool dyn = p.sched != nullptr && !p.dec_count;
+  const int m0 = p.n_mtiles ? *p.n_mtiles : p.cls[0].mtiles;
+  const int W0 = m0 * p.cls[0].ntiles * (p.cls[0].ksplit > 1 ? p.cls[0].ksplit : 1);
+  const int W = W0 + (p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0);
+  const bool dyn = p.sched != nullptr;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    int* segx = nullptr;  // concatenated decode mode: expert of each segment
-    if constexpr (BN == 16) {
-      if (p.dec_concat) {
-        segx = dec_seg_cache();
-        const int nseg = min(*p.dec_count, kDecodeMaxSegs);
-        for (int i = lane; i < nseg; i += 32) segx[i] = i ? p.dec.seg_expert[i] : 0;
-        __syncwarp();
-      }
-    }
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      // early_a: the B loads of the first STAGES stages wait for the
-      // previous launch; their coordinates are kept here meanwhile
-      bool early = early_a;
-      int pend_x[STAGES], pend_y[STAGES], pend_c[STAGES];
-      int npend = 0;
-      auto flush_pending = [&]() {
-        pdl_wait();
-        pdl_trigger();
-        for (int j = 0; j < npend; ++j)
-          tma_load_2d(tiles + j * Tr::kStageBytes + Tr::kABytes, &p.tmB[pend_c[j]], &full[j],
-                      pend_x[j], pend_y[j]);
-        early = false;
-      };
       // dynamic schedule: the next tile (the first is blockIdx.x) is taken
       // from the counter two k-blocks before the current tile's last load
       int nxt = int(blockIdx.x);
@@ -564,9 +306,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ring[slot] = w;
           mbar_arrive(&rfull[slot]);
           if (w < 0) break;
-          t = decode_tile<BN>(p, w, W0);
+          t = tile_at<BN>(p, w, W0);
           fetched = false;
-        } else if (!work_item<BN>(p, ds, W, W0, it, &t)) {
+        } else if (!work_item<BN>(p, W, W0, it, &t)) {
           break;
         }
         const GemmClass& C = p.cls[t.c];
@@ -586,38 +328,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = tiles + stage * Tr::kStageBytes;
           uint8_t* sb = sa + Tr::kABytes;
           mbar_arrive_expect_tx(&full[stage], Tr::kStageBytes);
-          int cls = t.c, arow = t.arow, brow = t.brow, kx = kb * bk;
-          if (segx) {  // k-block kb of the concatenation: segment sg, its block kk
-            const int sg = kb < ds.kbs ? 0 : 1 + (kb - ds.kbs) / ds.kbi;
-            const int kk = sg == 0 ? kb : kb - ds.kbs - (sg - 1) * ds.kbi;
-            cls = sg == 0 ? 1 : 0;
-            arow = sg == 0 ? t.row0 : segx[sg] * p.dec.M[0] + t.row0;
-            brow = sg * BN;  // 16 token rows per segment
-            kx = kk * 64;
-          }
+          const int kx = kb * bk;
           const int kbx = C.b_kwrap ? (kx % C.b_kwrap) : kx;
-          tma_load_2d(sa, &p.tmA[cls], &full[stage], kx, arow);
-          if (early) {
-            pend_x[npend] = kbx;
-            pend_y[npend] = brow;
-            pend_c[npend] = cls;
-            ++npend;
-          } else {
-            tma_load_2d(sb, &p.tmB[cls], &full[stage], kbx, brow);
-          }
+          tma_load_2d(sa, &p.tmA[t.c], &full[stage], kx, t.arow);
+          tma_load_2d(sb, &p.tmB[t.c], &full[stage], kbx, t.brow);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
-          if (early && npend == STAGES) flush_pending();
         }
         if (ok && !fetched) {
           nxt = int(gridDim.x) + atomicAdd(p.sched, 1);
           fetched = true;
         }
       }
-      if (early) flush_pending();
       if (!ok) {
         // Let the loads this thread issued land before the CTA exits: wait
         // (bounded, ignoring the abort flag) on the last min(issued, STAGES)
@@ -635,9 +360,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-    // (the producer warp's other lanes read nothing the previous launch
-    // writes and skip the wait: a blocking wait on the divergent path of
-    // the same warp could hold lane 0's early loads back)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -657,8 +379,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int w = ring[slot];
           mbar_arrive(&rempty[slot]);
           if (w < 0) break;
-          t = decode_tile<BN>(p, w, W0);
-        } else if (!work_item<BN>(p, ds, W, W0, it, &t)) {
+          t = tile_at<BN>(p, w, W0);
+        } else if (!work_item<BN>(p, W, W0, it, &t)) {
           break;
         }
         const bool f8 = p.cls[t.c].fp8 != 0;
@@ -724,8 +446,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!__shfl_sync(0xffffffffu, got, 0) || w < 0) break;
-        t = decode_tile<BN>(p, w, W0);
-      } else if (!work_item<BN>(p, ds, W, W0, it, &t)) {
+        t = tile_at<BN>(p, w, W0);
+      } else if (!work_item<BN>(p, W, W0, it, &t)) {
         break;
       }
       const GemmClass& C = p.cls[t.c];
@@ -740,9 +462,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int row = t.row0 + rloc;
       const bool rvalid = row < t.row_end;
 
-      if constexpr (BN == 16) {
-        decode_epilogue(p, ds, t, tb, rloc);
-      } else if (C.epi == EPI_TOPK) {
+      if (C.epi == EPI_TOPK) {
         router_epilogue<BN>(p, C, t, tb, row, rvalid);
       } else {
 #pragma unroll 1
@@ -869,14 +589,12 @@ cudaError_t prepare_impl() {
 
 cudaError_t prepare_grouped_gemm() {
   cudaError_t e;
-  if ((e = prepare_impl<16, 11>()) != cudaSuccess) return e;
   if ((e = prepare_impl<128, 6>()) != cudaSuccess) return e;
   return prepare_impl<256, 4>();
 }
 
 cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStream_t stream,
                                 bool pdl) {
-  if (bn == 16) return launch_impl<16, 11>(p, grid, stream, pdl);
   if (bn == 128) return launch_impl<128, 6>(p, grid, stream, pdl);
   if (bn == 256) return launch_impl<256, 4>(p, grid, stream, pdl);
   return cudaErrorInvalidValue;

@@ -763,8 +763,12 @@ moe_status moe_get_device_status(moe_handle* h, int32_t* status, void* stream) {
   MOE_TRY(cudaStreamSynchronize(s));
   if (*status != 0) {
     // A pass that gave up on a wait may have left its tile and schedule
-    // counters mid-count: start the next one from zero.
+    // counters mid-count, and partial sums in the decode accumulator: start
+    // the next one from zero.
     MOE_TRY(cudaMemsetAsync(h->dec.sync, 0, 4 * sizeof(unsigned), s));
+    MOE_TRY(cudaMemsetAsync(h->dec.acc, 0,
+                            size_t(moe::kDecodeMaxT) * h->cfg.hidden_size * sizeof(long long), s));
+    MOE_TRY(cudaMemsetAsync(h->dec.bad, 0, size_t(moe::kDecodeMaxT) * h->cfg.hidden_size, s));
     MOE_TRY(cudaMemsetAsync(h->sched, 0, 4 * sizeof(int32_t), s));
     MOE_TRY(cudaStreamSynchronize(s));
   }

@@ -21,46 +21,7 @@ enum EpiKind : int {
   EPI_F32 = 2,         // out = acc (float32)
   EPI_TOPK = 3,        // sigmoid top-k routing of the row (gate logits never stored)
   EPI_BLEND = 4,       // out = bf16(acc + blend_s + blend_res)  (LatentMoE fc2)
-  EPI_DEC_UP = 5,      // decode, weights x tokens: relu^2 (x routing weight) -> token-major rows
-  EPI_DEC_DOWN = 6,    // decode, weights x tokens: fp32 partial per piece, the last piece
-                       // of a 128-row output block sums them with the residual
 };
-
-// Decode tiles multiply 128 weight rows (A) by the <= 16 token vectors (B,
-// N = 16) of one segment: a routed expert slot or the shared expert.
-struct DecodeTile {
-  int cls;    // class (0 routed, 1 shared)
-  int seg;    // segment: 0 = shared expert, 1 + s = routed slot s
-  int arow;   // first A row (weight row, expert offset included)
-  int brow;   // first B row (token group)
-  int m0;     // first output row of the tile inside its segment's matrix
-};
-
-// Decode launches run a stream-K schedule: the k-blocks of all tiles, in
-// tile-list order (the n_first class-1 tiles first), are cut into equal
-// contiguous ranges, one per CTA; a piece is the part of one tile inside
-// one CTA's range.  Piece partials go to slot (tile + CTA index), so the
-// pieces of a tile occupy consecutive slots in k order.
-struct DecodeEpilogue {
-  int T;                       // tokens (<= 8)
-  int M[2];                    // output rows per class (I or S for up, H for down)
-  int n_first;                 // class-1 tiles at the head of the tile list
-  const float* seg_w;          // [segments, 16] routing weight of token t (0 if not routed)
-  __nv_bfloat16* out_up[2];    // up: [segments-or-1, 16, M] token-major relu^2 rows
-  float* up_part;              // up: [slots, 128, 16] partials of tiles cut into pieces
-  unsigned* up_counter;        // up: pieces finished per tile (self-resetting)
-  float* partial;              // down: [slots, 128, 16] piece partials
-  unsigned* mt_counter;        // down: pieces finished per 128-row tile (self-resetting)
-  const int* n_segments;       // down: segments of the step (device)
-  const int* seg_expert;       // down: expert of segment s >= 1 (device)
-  const __nv_bfloat16* residual;
-  __nv_bfloat16* hidden;       // [T, H]
-};
-
-// Smallest stream-K range (k-blocks) of a decode launch.
-constexpr int kDecMinPiece = 4;
-// Segments of a decode step: the shared expert plus at most T * k routed.
-constexpr int kDecodeMaxSegs = MOE_DECODE_MAX_TOKENS * MOE_MAX_TOP_K + 1;
 
 // Counts the kernels a call enqueues and, when profiling is enabled, records
 // caller-owned CUDA events around them: events[0] before the first launch,
@@ -133,23 +94,7 @@ struct GemmParams {
   const float* blend_s;
   const __nv_bfloat16* blend_res;
   int* status;
-  // Decode mode (BN = 16, dec_count non-null): tile i is dec_tiles[i] for
-  // i < *dec_count.
-  // With dec_concat (the down launch) the tiles are instead the 128-row
-  // output tiles, each over the concatenated K of all segments (shared
-  // expert first, then the routed slots in order), *dec_count is the number
-  // of segments, and the weight loads of the first stages are issued before
-  // waiting on the previous launch (they depend only on the routing, which
-  // is complete once the previous launch lets this one start).
-  const DecodeTile* dec_tiles;
-  const int* dec_count;
-  int dec_concat;
-  // Byte ranges prefetched into L2 while waiting on the previous launch
-  // (weights that do not depend on it); null = none.
-  const void* l2_prefetch[2];
-  size_t l2_prefetch_bytes[2];
-  DecodeEpilogue dec;
-  // Dynamic tile schedule (non-decode launches; null = static round-robin):
+  // Dynamic tile schedule (null = static round-robin):
   // sched[0] hands out tile indices past the first gridDim.x, sched[1]
   // counts exiting CTAs.  Both are zero before the launch and the last CTA
   // to exit zeroes them again.  Tiles are then taken shared class first
@@ -157,7 +102,7 @@ struct GemmParams {
   int* sched;
 };
 
-// Launch the persistent grouped GEMM (bn = 16, 128 or 256); the operand type
+// Launch the persistent grouped GEMM (bn = 128 or 256); the operand type
 // is a per-class property (GemmClass::fp8).  pdl: launch with programmatic
 // stream serialization (the kernel waits on griddepcontrol before reading
 // anything the previous kernel wrote).
