@@ -154,7 +154,8 @@ def test_committed_dram_captures_are_close_to_the_model():
         T = int(tok)
         s = WORKLOADS[name]
         path = "decode" if name == "decode" else "prefill"
-        U = s.k * T if path == "decode" else s.E  # T=1 decode: k experts; prefill: all
+        # touched experts: as captured (decode), all of them (prefill)
+        U = rec.get("distinct_experts", s.k * T) if path == "decode" else s.E
         model = dict((m[0], m) for m in bench.stage_model(s, T, path, U, router_split=True))
         stage_bytes = model[stage][1] if stage in model else model[stage.replace("_gemm", "_gemm_topk")][1]
         got = rec["dram_bytes_per_launch"]
