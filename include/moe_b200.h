@@ -125,6 +125,9 @@ typedef struct {
   const float* fc2_scale;         /* [H] f32, FP8 fc1 / fc2 only (else NULL) */
 } moe_weights;
 
+/* A layer instance.  Its workspace serves one forward at a time: calls on one
+ * handle are made from one host thread at a time, and passes enqueued on
+ * different streams must not overlap on the device. */
 typedef struct moe_handle moe_handle;
 
 /* Which implementation moe_forward_path runs. */
@@ -166,7 +169,11 @@ MOE_API moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual,
  * `stream`; the call returns after enqueueing them, so the caller
  * synchronises the stream before reading the host buffers.  Page-locked host
  * memory gives asynchronous copies.  Staging buffers come from the workspace
- * (no allocation). */
+ * (no allocation).  With at most MOE_DECODE_MAX_TOKENS tokens on the
+ * single-launch decode path, page-locked buffers that the device can address
+ * are written by the kernel itself (the output rows and the residual go over
+ * the bus as the kernel finishes them): one copy and one launch per call
+ * instead of up to three copies. */
 MOE_API moe_status moe_forward_host(moe_handle* h, void* hidden_host, void* residual_host,
                             int32_t num_tokens, void* stream);
 

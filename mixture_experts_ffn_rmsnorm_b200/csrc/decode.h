@@ -54,8 +54,9 @@ struct FusedDecodeArgs {
   const FusedWorkspace* ws;
   const CUtensorMap *tm_up, *tm_sup, *tm_down, *tm_sdown;  // weights as 128-row A boxes
   const CUtensorMap* tm_x[4];  // token rows, B boxes of 1, 2, 4, 8 rows (token-count bucket)
-  __nv_bfloat16* hidden;
-  __nv_bfloat16* residual;
+  __nv_bfloat16* hidden;    // [T, H] input rows
+  __nv_bfloat16* residual;  // [T, H] written with the input rows (device or mapped host memory)
+  __nv_bfloat16* out;       // [T, H] output rows (device or mapped host memory); null: hidden
   int T;
   int grid;
   int* status;

@@ -96,7 +96,7 @@ struct FusedParams {
   CUtensorMap tm_x;      // x16 [grid * 16, H]: 16 rows per CTA   (B, boxes of MAXT rows)
   const bf16* hidden;
   bf16* residual;
-  bf16* out;             // = hidden (written at the very end)
+  bf16* out;             // hidden (in place) or another buffer; written at the very end
   const bf16* norm_w;
   const bf16* gate_w;
   const float* gate_bias;
@@ -1051,7 +1051,7 @@ cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   p.tm_x = *a.tm_x[bucket];
   p.hidden = a.hidden;
   p.residual = a.residual;
-  p.out = a.hidden;
+  p.out = a.out ? a.out : a.hidden;
   p.norm_w = static_cast<const bf16*>(a.w->norm_w);
   p.gate_w = static_cast<const bf16*>(a.w->gate_w);
   p.gate_bias = a.w->gate_bias;

@@ -62,6 +62,19 @@ bool make_map(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner,
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The device address of page-locked host memory the device can address
+// (16-byte aligned), or null.
+void* mapped_device_pointer(const void* host) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || !a.devicePointer || !aligned16(a.devicePointer))
+    return nullptr;
+  return a.devicePointer;
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
@@ -528,8 +541,9 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
 
 // Decode path (T <= 8): one cooperative launch (decode_fused.cu) with the
 // weights as the 128-row operand and the tokens as N = 16.
+// out: where the output rows go (null: hidden, in place).
 moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cudaStream_t st,
-                          moe::LaunchLog* log) {
+                          moe::LaunchLog* log, bf16* out = nullptr) {
   const moe_config& c = h->cfg;
   if (!moe::fused_decode_supported(c, h->num_sms) || T < 1 || T > MOE_DECODE_MAX_TOKENS)
     return MOE_ERR_INVALID_CONFIG;
@@ -544,6 +558,7 @@ moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cu
   for (int b = 0; b < 4; ++b) a.tm_x[b] = &h->tm_dec_x[b];
   a.hidden = hidden;
   a.residual = residual;
+  a.out = out;
   a.T = T;
   a.grid = h->num_sms;
   a.status = h->status;
@@ -680,6 +695,25 @@ moe_status moe_forward_host(moe_handle* h, void* hidden_host, void* residual_hos
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t bytes = size_t(num_tokens) * h->cfg.hidden_size * sizeof(bf16);
   MOE_TRY(cudaMemcpyAsync(h->stage_h, hidden_host, bytes, cudaMemcpyHostToDevice, s));
+  // Decode sizes with page-locked buffers the device can address: the
+  // kernel writes the output rows (and the residual) into them itself, so
+  // no copy back and no launch of one follow the forward.
+  if (num_tokens <= MOE_DECODE_MAX_TOKENS && moe::fused_decode_supported(h->cfg, h->num_sms)) {
+    void* out_dev = mapped_device_pointer(hidden_host);
+    void* res_dev = out_dev && residual_host ? mapped_device_pointer(residual_host) : nullptr;
+    if (out_dev && (!residual_host || res_dev)) {
+      moe::LaunchLog log;
+      log.events = h->stage_events;
+      log.nevents = h->n_stage_events;
+      log.begin(s);
+      st = enqueue_decode(h, h->stage_h, res_dev ? static_cast<bf16*>(res_dev) : h->stage_r,
+                          num_tokens, s, &log, static_cast<bf16*>(out_dev));
+      h->last_launches = log.count;
+      h->last_tokens = num_tokens;
+      h->last_decode = true;
+      return st;
+    }
+  }
   st = moe_forward(h, h->stage_h, h->stage_r, num_tokens, stream);
   if (st != MOE_OK) return st;
   MOE_TRY(cudaMemcpyAsync(hidden_host, h->stage_h, bytes, cudaMemcpyDeviceToHost, s));
