@@ -270,32 +270,58 @@ __device__ __forceinline__ bool step_of(const Units& u, int m, int s, int* kind,
 // the factor r_t = rsqrt(mean x_t^2 + eps), so it needs nothing but the
 // loads; the epilogue applies r_t to accumulator column t instead
 // (W . (x r w) = r (W . (x w))).
+//
+// One or two tokens: every chunk's loads are in flight at once, issued
+// first of all, before the launch's set-up (route_issue): the routing
+// decides when the routed weights can stream, and the set-up's cold
+// instruction fetches then overlap the loads' DRAM latency (2.5 us earlier
+// routing at T = 1).  More tokens would spill those registers: their chunks
+// go one at a time, in route_logits (issuing the first one early was
+// slower at T = 8).
 template <int MAXT>
-__device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
+struct RouteLoads {
+  static constexpr bool kHold = MAXT <= 2;
+  static constexpr int kHeld = kHold ? kMaxChunks : 1;
+  uint4 x[kHeld][MAXT], w[kHeld], a[kHeld], b[kHeld];
+};
+
+// Chunk j of routing thread rt: the norm weight, this CTA's gate rows and
+// the tokens, 8 elements each.
+template <int MAXT>
+__device__ __forceinline__ void route_load_chunk(const FusedParams& p, int rt, int j,
+                                                 uint4 (&x)[MAXT], uint4& w, uint4& a, uint4& b) {
+  const int H = p.H, E = p.E, G = gridDim.x;
+  const int e0 = blockIdx.x, e1 = blockIdx.x + G;
+  const int c = rt + j * kRouteThreads;
+  const bool in = c < H / 8;
+  w = in ? __ldg(reinterpret_cast<const uint4*>(p.norm_w) + c) : make_uint4(0, 0, 0, 0);
+  a = in && e0 < E ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e0) * H) + c)
+                   : make_uint4(0, 0, 0, 0);
+  b = in && e1 < E ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e1) * H) + c)
+                   : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int t = 0; t < MAXT; ++t)
+    x[t] = in && t < p.T ? reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c]
+                         : make_uint4(0, 0, 0, 0);
+}
+
+template <int MAXT>
+__device__ __forceinline__ void route_issue(const FusedParams& p, int rt, RouteLoads<MAXT>& L) {
+  if constexpr (RouteLoads<MAXT>::kHold) {
+#pragma unroll
+    for (int j = 0; j < kMaxChunks; ++j)
+      route_load_chunk<MAXT>(p, rt, j, L.x[j], L.w[j], L.a[j], L.b[j]);
+  }
+}
+
+template <int MAXT>
+__device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoads<MAXT>& L) {
   const int H = p.H, T = p.T, E = p.E, G = gridDim.x;
   const int nv = H / 8;
   const int warp = rt >> 5, lane = rt & 31;
   const int e0 = blockIdx.x, e1 = blockIdx.x + G;
   const bool has0 = e0 < E, has1 = e1 < E;
   bf16* x16 = p.ws.x16 + size_t(blockIdx.x) * kDecodeN * H;
-  // One or two tokens: every chunk's loads in flight at once.  More tokens
-  // would spill those registers: their chunks go one at a time.
-  constexpr bool kHold = MAXT <= 2;
-  constexpr int kHeld = kHold ? kMaxChunks : 1;
-  uint4 xv[kHeld][MAXT], wv[kHeld], g0[kHeld], g1[kHeld];
-  auto load_chunk = [&](int j, uint4 (&x)[MAXT], uint4& w, uint4& a, uint4& b) {
-    const int c = rt + j * kRouteThreads;
-    const bool in = c < nv;
-    w = in ? __ldg(reinterpret_cast<const uint4*>(p.norm_w) + c) : make_uint4(0, 0, 0, 0);
-    a = in && has0 ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e0) * H) + c)
-                   : make_uint4(0, 0, 0, 0);
-    b = in && has1 ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e1) * H) + c)
-                   : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int t = 0; t < MAXT; ++t)
-      x[t] = in && t < T ? reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c]
-                         : make_uint4(0, 0, 0, 0);
-  };
   float ss[MAXT], d0[MAXT], d1[MAXT];
 #pragma unroll
   for (int t = 0; t < MAXT; ++t) ss[t] = d0[t] = d1[t] = 0.f;
@@ -330,16 +356,14 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt) {
       }
     }
   };
-  if constexpr (kHold) {
+  if constexpr (RouteLoads<MAXT>::kHold) {
 #pragma unroll
-    for (int j = 0; j < kMaxChunks; ++j) load_chunk(j, xv[j], wv[j], g0[j], g1[j]);
-#pragma unroll
-    for (int j = 0; j < kMaxChunks; ++j) consume(j, xv[j], wv[j], g0[j], g1[j]);
+    for (int j = 0; j < kMaxChunks; ++j) consume(j, L.x[j], L.w[j], L.a[j], L.b[j]);
   } else {
 #pragma unroll 1
     for (int j = 0; j < kMaxChunks; ++j) {
-      load_chunk(j, xv[0], wv[0], g0[0], g1[0]);
-      consume(j, xv[0], wv[0], g0[0], g1[0]);
+      route_load_chunk<MAXT>(p, rt, j, L.x[0], L.w[0], L.a[0], L.b[0]);
+      consume(j, L.x[0], L.w[0], L.a[0], L.b[0]);
     }
   }
   if (rt < E) sh.bias[rt] = p.gate_bias ? p.gate_bias[rt] : 0.f;
@@ -409,6 +433,31 @@ __device__ __noinline__ bool route_select(const FusedParams& p, Shared& sh, int 
     }
     named_barrier(bar, kRouteThreads);
     if (sh.route_fail) return false;
+  }
+  if (T == 1) {
+    // One token: its k choices are distinct experts, and slot s is choice s.
+    // One warp does it all (no table scan, no further barriers but the last).
+    if (warp == 0) {
+      warp_topk(p.ws.logits, p.gate_bias ? sh.bias : nullptr, E, k, p.rsf, sh.sel_idx, sh.sel_w);
+      for (int i = lane; i < k * kDecodeN; i += 32) (&sh.seg_w[0][0])[i] = 0.f;
+      __syncwarp();
+      if (lane < k) {
+        const int e = sh.sel_idx[lane];
+        const float w = sh.sel_w[lane];
+        if (!dry && blockIdx.x == 0) {  // the routing of the pass, for moe_copy_routing
+          p.ws.idx[lane] = e;
+          p.ws.w[lane] = w;
+        }
+        // an id outside [0, E) (only from NaN logits) is routed nowhere
+        const bool valid = unsigned(e) < unsigned(E);
+        sh.seg_expert[lane] = valid ? e : 0;
+        if (valid) sh.seg_w[lane][0] = w;
+        if (!valid && !dry) atomicOr(p.status, kStatusBadIndex);
+      }
+      if (lane == 0) sh.U = k;
+    }
+    named_barrier(bar, kRouteThreads);
+    return true;
   }
   for (int t = warp; t < T; t += 4)
     warp_topk(p.ws.logits + t * E, p.gate_bias ? sh.bias : nullptr, E, k, p.rsf,
@@ -574,6 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   un.nS = (p.S + kBM - 1) / kBM;
   un.nI = (p.I + kBM - 1) / kBM;
   un.N = un.nS;  // the routed units are added once the routing is known
+
+  RouteLoads<MAXT> rl;
+  if (warp >= 6) route_issue<MAXT>(p, threadIdx.x - 192, rl);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -967,7 +1019,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   } else {
     // ------------------------------------------------------------- routing
     const int rt = threadIdx.x - 192;
-    route_logits<MAXT>(p, sh, rt);
+    route_logits<MAXT>(p, sh, rt, rl);
     route_select(p, sh, rt, abort, kBarRoute, false);
     if (rt == 0) mbar_arrive(&sh.routed);  // (also on failure: the waiters then see abort)
   }
