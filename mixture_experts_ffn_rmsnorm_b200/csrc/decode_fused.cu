@@ -406,6 +406,20 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoad
   }
 }
 
+// The sigmoid top-k of token t by one warp, into sel_idx / sel_w.  The dry
+// pass (see route_select) loads no logits: it must only run the same
+// instructions, and a load from DRAM would hold it up.
+__device__ __forceinline__ void topk_of_token(const FusedParams& p, Shared& sh, int t, int lane,
+                                              bool dry) {
+  const int E = p.E;
+  float lg[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    lg[j] = !dry && lane + 32 * j < E ? __ldcg(p.ws.logits + t * E + lane + 32 * j) : 0.f;
+  warp_topk_regs(lg, p.gate_bias ? sh.bias : nullptr, E, p.k, p.rsf, sh.sel_idx + t * p.k,
+                 sh.sel_w + t * p.k);
+}
+
 // Once every CTA's logits are in: the sigmoid top-k of every token and the
 // routed slot table (identical in every CTA).  Returns false on timeout.
 //
@@ -438,7 +452,7 @@ __device__ __noinline__ bool route_select(const FusedParams& p, Shared& sh, int 
     // One token: its k choices are distinct experts, and slot s is choice s.
     // One warp does it all (no table scan, no further barriers but the last).
     if (warp == 0) {
-      warp_topk(p.ws.logits, p.gate_bias ? sh.bias : nullptr, E, k, p.rsf, sh.sel_idx, sh.sel_w);
+      topk_of_token(p, sh, 0, lane, dry);
       for (int i = lane; i < k * kDecodeN; i += 32) (&sh.seg_w[0][0])[i] = 0.f;
       __syncwarp();
       if (lane < k) {
@@ -459,9 +473,7 @@ __device__ __noinline__ bool route_select(const FusedParams& p, Shared& sh, int 
     named_barrier(bar, kRouteThreads);
     return true;
   }
-  for (int t = warp; t < T; t += 4)
-    warp_topk(p.ws.logits + t * E, p.gate_bias ? sh.bias : nullptr, E, k, p.rsf,
-              sh.sel_idx + t * k, sh.sel_w + t * k);
+  for (int t = warp; t < T; t += 4) topk_of_token(p, sh, t, lane, dry);
   for (int i = rt; i < kMaxSlots * kDecodeN; i += kRouteThreads) (&sh.seg_w[0][0])[i] = 0.f;
   named_barrier(bar, kRouteThreads);
   const int R = T * k;
