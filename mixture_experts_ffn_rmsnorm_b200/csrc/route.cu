@@ -277,11 +277,26 @@ __global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ u,
   const float inv = 1.f / s;
   const uint4* src = reinterpret_cast<const uint4*>(x + size_t(p) * W);
   uint2* dst = reinterpret_cast<uint2*>(q + size_t(p) * W);
-  for (int i = threadIdx.x; i < W / 8; i += blockDim.x) {
-    float f[8];
-    unpack8(src[i], f);
-    dst[i] = make_uint2(e4m3x4(f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv),
-                        e4m3x4(f[4] * inv, f[5] * inv, f[6] * inv, f[7] * inv));
+  // kBatch chunks of 8 per thread in flight before the first conversion
+  constexpr int kBatch = 4;
+  const int nv = W / 8;
+  for (int i0 = threadIdx.x; i0 < nv; i0 += kBatch * blockDim.x) {
+    uint4 xv[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int i = i0 + b * blockDim.x;
+      if (i < nv) xv[b] = __ldcs(src + i);
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int i = i0 + b * blockDim.x;
+      if (i < nv) {
+        float f[8];
+        unpack8(xv[b], f);
+        dst[i] = make_uint2(e4m3x4(f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv),
+                            e4m3x4(f[4] * inv, f[5] * inv, f[6] * inv, f[7] * inv));
+      }
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -433,7 +448,18 @@ __global__ void gather_kernel(const uint8_t* __restrict__ X, size_t ldx,
   const int t = perm[p] / k;
   const uint4* src = reinterpret_cast<const uint4*>(X + size_t(t) * ldx);
   uint4* dst = reinterpret_cast<uint4*>(xs + size_t(p) * row_bytes);
-  for (int i = lane; i < row_bytes / 16; i += 32) dst[i] = src[i];
+  // kBatch loads per lane in flight before the first store
+  constexpr int kBatch = 4;
+  const int nv = row_bytes / 16;
+  for (int i0 = lane; i0 < nv; i0 += kBatch * 32) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      if (i0 + b * 32 < nv) v[b] = src[i0 + b * 32];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      if (i0 + b * 32 < nv) dst[i0 + b * 32] = v[b];
+  }
   if (scale && lane == 0) xs_scale[p] = scale[t];
 }
 
