@@ -132,8 +132,11 @@ typedef struct moe_handle moe_handle;
 
 /* Which implementation moe_forward_path runs. */
 typedef enum {
-  MOE_PATH_AUTO = 0,     /* decode path for num_tokens <= MOE_DECODE_MAX_TOKENS, else prefill */
-  MOE_PATH_DECODE = 1,   /* weight-streaming tensor-core decode, weights x tokens (num_tokens <= MOE_DECODE_MAX_TOKENS) */
+  MOE_PATH_AUTO = 0,     /* the decode path for num_tokens <= MOE_DECODE_MAX_TOKENS (with FP8 routed
+                            experts: num_tokens == 1) where the layer supports it, else prefill */
+  MOE_PATH_DECODE = 1,   /* weight-streaming tensor-core decode in one launch, weights x tokens
+                            (num_tokens <= MOE_DECODE_MAX_TOKENS; direct layers with a BF16 shared
+                            expert; FP8 routed experts are dequantised in shared memory) */
   MOE_PATH_PREFILL = 2   /* sort by expert + tcgen05 grouped GEMMs (any num_tokens) */
 } moe_path;
 

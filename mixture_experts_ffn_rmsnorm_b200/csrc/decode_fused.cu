@@ -38,6 +38,9 @@
 //
 // Every wait is bounded (about one second): a timeout sets a status bit, the
 // CTA drains its own TMA loads and MMAs, frees its TMEM and returns.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "decode.h"
 #include "ptx.cuh"
 #include "topk.cuh"
@@ -57,6 +60,22 @@ constexpr int kStages = 5;
 constexpr int kABytes = kBM * 128;          // 128 weight rows x 64 BF16
 constexpr int kBBytes = kDecodeN * 128;     // 16 token rows x 64 BF16
 constexpr int kStageBytes = kKB * (kABytes + kBBytes);
+// FP8 routed experts (E4M3 weights, one fp32 scale per weight row): the
+// weights stream as FP8 boxes of 128 rows x 128 bytes (= one stage's two
+// 64-wide k-blocks) into kF8Slots staging slots, with the up GEMM's token
+// boxes beside them; the routing warps, idle once the routing is done,
+// dequantise each box (value x its row's scale, rounded to BF16) into a BF16
+// stage that the MMA reads as before.  Those CTAs keep kStagesF8 BF16
+// stages.  The CTAs of the (BF16) shared expert use the same memory as
+// kStages BF16 stages.
+constexpr int kStagesF8 = 2;
+constexpr int kF8Slots = 6;
+constexpr int kF8ABytes = kBM * 128;              // 128 rows x 128 E4M3
+constexpr int kF8SlotBytes = kF8ABytes + kKB * kBBytes;
+constexpr int kRingBytesF8 = kStagesF8 * kStageBytes + kF8Slots * kF8SlotBytes;
+constexpr int kRingBytes(bool f8) {
+  return f8 && kRingBytesF8 > kStages * kStageBytes ? kRingBytesF8 : kStages * kStageBytes;
+}
 constexpr int kUBytes = 2 * kBBytes;        // a unit's relu^2 rows: 16 tokens x 128 K, two 64-wide chunks
 constexpr int kThreads = 320;               // see the warp roles above
 constexpr int kEpiThreads = 128;
@@ -65,7 +84,7 @@ constexpr int kMaxSlots = kDecodeMaxT * kTopKMax;  // routed slots (distinct exp
 constexpr int kMaxChunks = 4;               // 8-element chunks per routing thread (H <= 4096)
 constexpr int kTmemCols = 512;              // 2 x 16 (up) + ceil(H / 128) x 16 (down)
 constexpr int kMaxRowTiles = kTmemCols / kDecodeN - 2;
-constexpr int kSmem = kStages * kStageBytes + 2 * kUBytes + 1024 + 1024;
+constexpr int kSmemOf(bool f8) { return kRingBytes(f8) + 2 * kUBytes + 1024 + 1024; }
 
 // Output rows that each CTA finishes: ceil(H / grid), rounded up to a
 // multiple of 4 (vector loads and stores).
@@ -100,6 +119,8 @@ struct FusedParams {
   const bf16* norm_w;
   const bf16* gate_w;
   const float* gate_bias;
+  const float* up_scale;    // [E, I] FP8 routed experts' row scales (else null)
+  const float* down_scale;  // [E, H]
   int T, H, E, k, I, S;
   float eps, rsf;
   FusedWorkspace ws;
@@ -164,6 +185,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -173,6 +199,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Shared state of one CTA.
 struct Shared {
   uint64_t full[kStages], empty[kStages];
+  uint64_t f8full[kF8Slots], f8empty[kF8Slots];  // FP8 staging slots: TMA -> dequantisation
   uint64_t tfull[2], tempty[2];   // up accumulators: MMA -> epilogue -> MMA
   uint64_t ufull[2], ufree[2];    // relu^2 row buffers: epilogue -> MMA -> epilogue
   uint64_t down_done;             // every down MMA of the CTA has completed
@@ -185,6 +212,7 @@ struct Shared {
   int abort;
   int stop;                 // the epilogue warps' common decision to stop (epi_stop)
   int route_fail;
+  int conv_stop;            // the dequantising warps' common decision to stop
   int flag;
   int U;                    // routed slots
   float rs[kDecodeMaxT];
@@ -198,7 +226,9 @@ struct Shared {
   float bias[MOE_MAX_EXPERTS];
 };
 
-static_assert(kSmem + sizeof(Shared) <= 227 * 1024, "shared memory of one CTA");
+static_assert(kSmemOf(false) + sizeof(Shared) <= 227 * 1024, "shared memory of one CTA");
+static_assert(kSmemOf(true) + sizeof(Shared) <= 227 * 1024, "shared memory of one CTA (FP8)");
+static_assert(kStagesF8 <= kStages, "barrier arrays");
 
 // The four epilogue warps meet here and take one decision together:
 // whether to stop (some role recorded a timeout).  Control flow of the
@@ -212,15 +242,27 @@ __device__ __forceinline__ bool epi_stop(Shared& sh, int tid) {
 
 // ------------------------------------------------------------------ units
 // Units: shared-expert tiles j < nS, then routed tile (j - nS) % nI of slot
-// (j - nS) / nI.  CTA c takes j = c, c + grid, c + 2 grid, ...  Its steps:
+// (j - nS) / nI.  CTA c takes j = c, c + grid, c + 2 grid, ...  With FP8
+// routed experts the two kinds stay on separate CTAs (a CTA's stages are
+// either BF16 or FP8): CTA c < nS takes shared unit c alone, and the routed
+// units go round-robin over the other Gr = grid - nS CTAs.  Its steps:
 // the up of each unit and the down of each unit, ordered so that a unit's
 // down comes one unit after its up (the relu^2 rows are ready by then),
 // except that a shared first unit is followed by its own down at once (its
 // successors wait for the routing).
 struct Units {
   int c, G, nS, nI, N;  // N = nS + U * nI, the units of the pass (known after routing)
-  __device__ __forceinline__ int count() const { return c < N ? (N - 1 - c) / G + 1 : 0; }
-  __device__ __forceinline__ int unit(int n) const { return c + n * G; }
+  bool f8;              // FP8 routed experts: shared and routed units on separate CTAs
+  __device__ __forceinline__ int count() const {
+    if (!f8) return c < N ? (N - 1 - c) / G + 1 : 0;
+    if (c < nS) return 1;
+    const int r = c - nS, nr = N - nS, Gr = G - nS;
+    return r < nr ? (nr - 1 - r) / Gr + 1 : 0;
+  }
+  __device__ __forceinline__ int unit(int n) const {
+    if (!f8) return c + n * G;
+    return c < nS ? c : c + n * (G - nS);
+  }
   __device__ __forceinline__ bool shared_first() const { return c < nS; }
 };
 
@@ -314,8 +356,11 @@ __device__ __forceinline__ void route_issue(const FusedParams& p, int rt, RouteL
   }
 }
 
+// f16tok: write the token rows as f16 instead of BF16 (the up GEMM of FP8
+// units runs on f16 operands).
 template <int MAXT>
-__device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoads<MAXT>& L) {
+__device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoads<MAXT>& L,
+                             bool f16tok) {
   const int H = p.H, T = p.T, E = p.E, G = gridDim.x;
   const int nv = H / 8;
   const int warp = rt >> 5, lane = rt & 31;
@@ -350,8 +395,14 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoad
       }
       if (c < nv && t < T) {
         reinterpret_cast<uint4*>(x16 + size_t(t) * H)[c] =
-            make_uint4(pack_bf16x2(f[0] * w[0], f[1] * w[1]), pack_bf16x2(f[2] * w[2], f[3] * w[3]),
-                       pack_bf16x2(f[4] * w[4], f[5] * w[5]), pack_bf16x2(f[6] * w[6], f[7] * w[7]));
+            f16tok ? make_uint4(pack_f16x2(f[0] * w[0], f[1] * w[1]),
+                                pack_f16x2(f[2] * w[2], f[3] * w[3]),
+                                pack_f16x2(f[4] * w[4], f[5] * w[5]),
+                                pack_f16x2(f[6] * w[6], f[7] * w[7]))
+                   : make_uint4(pack_bf16x2(f[0] * w[0], f[1] * w[1]),
+                                pack_bf16x2(f[2] * w[2], f[3] * w[3]),
+                                pack_bf16x2(f[4] * w[4], f[5] * w[5]),
+                                pack_bf16x2(f[6] * w[6], f[7] * w[7]));
         if (blockIdx.x == 0) reinterpret_cast<uint4*>(p.residual + size_t(t) * H)[c] = x[t];
       }
     }
@@ -569,6 +620,59 @@ __device__ __forceinline__ UnitInfo unit_info(const FusedParams& p, const Shared
 // of an expert may have only 64 valid rows).
 __device__ __forceinline__ int down_kk(const UnitInfo& f) { return f.rows - f.row0 >= kBM ? 2 : 1; }
 
+// ------------------------------------------------------ FP8 dequantisation
+// Row r of FP8 staging slot f8 (128 rows x 128 E4M3, 128-byte swizzle: the
+// 16-byte chunk j of row r sits at j ^ (r % 8)) into BF16-layout stage st:
+// its two 64-wide k-blocks, same swizzle, zeros for a row outside the
+// matrix.
+//   up:   f16, exactly the E4M3 values (every E4M3 value is an f16); the
+//         row's scale is applied to the accumulator row in the epilogue, and
+//         the tokens are f16 too.  The thread also copies its 32 bytes of
+//         the two token boxes.
+//   down: BF16 of the value times the row's scale (the product in f16,
+//         rounded once more to BF16): the down accumulator adds units of
+//         different experts, so each weight row carries its own scale.
+template <bool UP>
+__device__ __forceinline__ void dequant_row(const uint8_t* f8, uint8_t* st, int r, float scale,
+                                            bool valid) {
+  const uint8_t* src = f8 + r * 128;
+  const __half2 s2 = __float2half2_rn(scale);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint4 q = *reinterpret_cast<const uint4*>(src + ((j ^ (r & 7)) << 4));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      __half2 lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[h] & 0xFFFFu),
+                                              __NV_E4M3);
+      __half2 hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[h] >> 16),
+                                              __NV_E4M3);
+      if constexpr (UP) {
+        o[2 * h] = valid ? *reinterpret_cast<uint32_t*>(&lo) : 0u;
+        o[2 * h + 1] = valid ? *reinterpret_cast<uint32_t*>(&hi) : 0u;
+      } else {
+        const float2 a = __half22float2(__hmul2(lo, s2)), b = __half22float2(__hmul2(hi, s2));
+        o[2 * h] = valid ? pack_bf16x2(a.x, a.y) : 0u;
+        o[2 * h + 1] = valid ? pack_bf16x2(b.x, b.y) : 0u;
+      }
+    }
+    // E4M3 elements 16 j .. 16 j + 15 are chunks 2 (j % 4) and 2 (j % 4) + 1
+    // of k-block j / 4
+    uint8_t* dst = st + (j >> 2) * kABytes + r * 128;
+    const int c0 = (j & 3) * 2;
+    *reinterpret_cast<uint4*>(dst + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + (((c0 + 1) ^ (r & 7)) << 4)) =
+        make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  if constexpr (UP) {
+    const uint4* tb = reinterpret_cast<const uint4*>(f8 + kF8ABytes) + 2 * r;
+    uint4* db = reinterpret_cast<uint4*>(st + kKB * kABytes) + 2 * r;
+    db[0] = tb[0];
+    db[1] = tb[1];
+  }
+}
+
 // ------------------------------------------------------------ reduction
 // Adds this CTA's partial value v of output element `at` (token-major
 // [T, H]) into the fixed-point accumulator.
@@ -616,13 +720,94 @@ __device__ __noinline__ void finish_slice(const FusedParams& p, int T, int r0, i
   }
 }
 
+// The routing warps' second job in a CTA with FP8 routed units: every stage
+// of the CTA's steps, in the producer's and the MMA's order, from its FP8
+// staging slot into the next BF16 stage (which the MMA frees), then the
+// stage to the MMA and the slot back to the producer.  Returns false on a
+// timeout (recorded).
+__device__ bool dequant_stages(const FusedParams& p, Shared& sh, const Units& un, uint8_t* tiles,
+                               int rt, volatile int* abort) {
+  const int kbH = p.H / 64, nH = (p.H + kBM - 1) / kBM;
+  uint8_t* slots = tiles + kStagesF8 * kStageBytes;
+  int st = 0, fs = 0;
+  uint32_t sph = 0, fph = 0;
+  const int m = un.count();
+  for (int s = 0;; ++s) {
+    int kind, n;
+    if (!step_of(un, m, s, &kind, &n)) break;
+    const UnitInfo f = unit_info(p, sh, un, n);
+    const int nstage = kind == 0 ? (kbH + kKB - 1) / kKB : nH;
+    // down: this thread's row scales for the whole step (one per 128-row
+    // block of the output, row i * 128 + rt), loaded before its first stage
+    // (a scale load per stage would put a memory round trip into every
+    // stage); up needs none here (the epilogue applies them)
+    float sc[kMaxRowTiles];
+#pragma unroll
+    for (int i = 0; i < kMaxRowTiles; ++i) {
+      const int row = i * kBM + rt;
+      sc[i] = kind == 1 && i < nH && row < p.H ? p.down_scale[size_t(f.expert) * p.H + row]
+                                               : 0.f;
+    }
+#pragma unroll 1
+    for (int i = 0; i < nstage; ++i) {
+      // one thread waits (bounded) for the slot's data and the stage's
+      // room, then all take its decision together (no thread may leave a
+      // named barrier's count short)
+      if (rt == 0) {
+        const bool ok = mbar_wait(&sh.f8full[fs], fph, abort) &&
+                        mbar_wait(&sh.empty[st], sph ^ 1u, abort);
+        if (!ok) record_timeout(p.status, abort);
+        sh.conv_stop = !ok;
+      }
+      named_barrier(kBarRoute, kRouteThreads);
+      if (sh.conv_stop) return false;
+      // (both phases are complete: every thread observes them itself)
+      mbar_wait(&sh.f8full[fs], fph, abort);
+      mbar_wait(&sh.empty[st], sph ^ 1u, abort);
+      // up: weight row = intermediate row f.row0 + rt of the expert; down:
+      // weight row = output row i * 128 + rt
+      bool valid;
+      float scale;
+      if (kind == 0) {
+        valid = f.row0 + rt < f.rows;
+        scale = 1.f;
+      } else {
+        valid = i * kBM + rt < p.H;
+        scale = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxRowTiles; ++j)
+          if (j == i) scale = sc[j];
+      }
+      if (kind == 0)
+        dequant_row<true>(slots + fs * kF8SlotBytes, tiles + st * kStageBytes, rt, scale, valid);
+      else
+        dequant_row<false>(slots + fs * kF8SlotBytes, tiles + st * kStageBytes, rt, scale, valid);
+      fence_proxy_async_shared();  // generic writes -> tensor core reads
+      named_barrier(kBarRoute, kRouteThreads);
+      if (rt == 0) {
+        mbar_arrive(&sh.full[st]);
+        mbar_arrive(&sh.f8empty[fs]);
+      }
+      if (++st == kStagesF8) {
+        st = 0;
+        sph ^= 1u;
+      }
+      if (++fs == kF8Slots) {
+        fs = 0;
+        fph ^= 1u;
+      }
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- kernel
-template <int MAXT>
+template <int MAXT, bool F8>
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ FusedParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* tiles = smem_raw + pad;
-  uint8_t* ubufs = tiles + kStages * kStageBytes;  // two relu^2 row buffers
+  uint8_t* ubufs = tiles + kRingBytes(F8);  // two relu^2 row buffers
   Shared& sh = *reinterpret_cast<Shared*>(ubufs + 2 * kUBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -635,6 +820,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   un.nS = (p.S + kBM - 1) / kBM;
   un.nI = (p.I + kBM - 1) / kBM;
   un.N = un.nS;  // the routed units are added once the routing is known
+  un.f8 = F8;
+  // this CTA's units are FP8 (dequantised by the routing warps), and the
+  // BF16 stages it has
+  const bool conv = F8 && cta >= un.nS;
+  const int nst = conv ? kStagesF8 : kStages;
 
   RouteLoads<MAXT> rl;
   if (warp >= 6) route_issue<MAXT>(p, threadIdx.x - 192, rl);
@@ -656,6 +846,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     mbar_init(&sh.routed, 1);
     mbar_init(&sh.warm, 1);
     mbar_init(&sh.drain, 1);
+    if (F8) {
+      for (int s = 0; s < kF8Slots; ++s) {
+        mbar_init(&sh.f8full[s], 1);
+        mbar_init(&sh.f8empty[s], 1);
+      }
+    }
     sh.abort = 0;
     sh.U = 0;
     fence_barrier_init();
@@ -756,6 +952,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         }
         return true;
       };
+      // FP8 units: one E4M3 weight box (two k-blocks; for up also the two
+      // token boxes) into the next free staging slot, for the routing warps
+      // to dequantise
+      uint8_t* slots = tiles + kStagesF8 * kStageBytes;
+      int fs = 0, issued8 = 0;
+      uint32_t fph = 0;
+      bool tok8 = false;
+      auto issue8 = [&](const CUtensorMap* map, int ax, int ay, bool up, int bx) -> bool {
+        if (!mbar_wait(&sh.f8empty[fs], fph ^ 1u, abort)) {
+          record_timeout(p.status, abort);
+          return false;
+        }
+        if (up && !tok8) {  // (complete since the routing; makes the rows visible to TMA)
+          if (!mbar_wait(&sh.tokens, 0, abort)) {
+            record_timeout(p.status, abort);
+            return false;
+          }
+          fence_proxy_async_global();
+          tok8 = true;
+        }
+        uint8_t* sl = slots + fs * kF8SlotBytes;
+        mbar_arrive_expect_tx(&sh.f8full[fs], uint32_t(kF8ABytes + (up ? kKB * MAXT * 128 : 0)));
+        tma_load_2d_hint(sl, map, &sh.f8full[fs], ax, ay, stream_policy);
+        if (up)
+          for (int i = 0; i < kKB; ++i)
+            tma_load_2d(sl + kF8ABytes + i * kBBytes, &p.tm_x, &sh.f8full[fs], bx + i * 64, xrow);
+        ++issued8;
+        if (++fs == kF8Slots) {
+          fs = 0;
+          fph ^= 1u;
+        }
+        return true;
+      };
       int m = 0;
       bool routed = false;
       for (int s = 0; ok; ++s) {
@@ -786,7 +1015,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           if (!step_of(un, m, s, &kind, &n)) break;
         }
         const UnitInfo f = unit_info(p, sh, un, n);
-        if (kind == 0) {  // up: W_up[rows] x tokens, K = H
+        if (conv) {  // FP8 routed unit (E4M3 boxes of 128 elements = two k-blocks)
+          if (kind == 0) {
+            for (int kb = 0; ok && kb < kbH; kb += kKB)
+              ok = issue8(&p.tm_up, kb * 64, f.expert * p.I + f.row0, true, kb * 64);
+          } else {
+            for (int r = 0; ok && r < nH; ++r)
+              ok = issue8(&p.tm_down, f.row0, f.expert * p.H + r * kBM, false, 0);
+          }
+        } else if (kind == 0) {  // up: W_up[rows] x tokens, K = H
           const CUtensorMap* map = f.shared ? &p.tm_sup : &p.tm_up;
           const int ay = f.shared ? f.row0 : f.expert * p.I + f.row0;
           for (int kb = 0; ok && kb < kbH; kb += kKB)
@@ -824,12 +1061,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           int zero = 0;
           mbar_wait(&sh.full[s], ph, &zero);
         }
+        // and the FP8 boxes in flight
+        s = fs;
+        ph = fph;
+        const int n8 = issued8 < kF8Slots ? issued8 : kF8Slots;
+        for (int i = 0; i < n8; ++i) {
+          if (--s < 0) {
+            s = kF8Slots - 1;
+            ph ^= 1u;
+          }
+          int zero = 0;
+          mbar_wait(&sh.f8full[s], ph, &zero);
+        }
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(kBM, kDecodeN, 1, 1);  // BF16 x BF16 -> F32
+      const uint32_t idesc = make_idesc(kBM, kDecodeN, 1, 1);    // BF16 x BF16 -> F32
+      const uint32_t idesc_h = make_idesc(kBM, kDecodeN, 0, 0);  // F16 x F16 -> F32 (FP8 units' up)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -877,11 +1127,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t koff = uint64_t((kk * 32) >> 4);
-                umma_f16(d, ad + koff, bd + koff, idesc, (kb + i != 0 || kk != 0) ? 1u : 0u);
+                umma_f16(d, ad + koff, bd + koff, conv ? idesc_h : idesc,
+                         (kb + i != 0 || kk != 0) ? 1u : 0u);
               }
             }
             umma_commit(&sh.empty[stage]);
-            if (++stage == kStages) {
+            if (++stage == nst) {
               stage = 0;
               phase ^= 1u;
             }
@@ -916,7 +1167,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
               }
             }
             umma_commit(&sh.empty[stage]);
-            if (++stage == kStages) {
+            if (++stage == nst) {
               stage = 0;
               phase ^= 1u;
             }
@@ -966,6 +1217,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       const UnitInfo f = unit_info(p, sh, un, n);
       const int b = n & 1;
       const uint32_t par = (n >> 1) & 1;
+      const bool valid = f.row0 + rloc < f.rows;
+      // an FP8 unit's up runs on the unscaled E4M3 values: its row's scale
+      // (loaded while the up runs)
+      const float srow = conv && !f.shared && valid
+                             ? p.up_scale[size_t(f.expert) * p.I + f.row0 + rloc]
+                             : 1.f;
       // the up accumulator of unit n
       if (lane == 0 && !mbar_wait(&sh.tfull[b], par, abort)) record_timeout(p.status, abort);
       __syncwarp();
@@ -983,11 +1240,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       // relu^2 times the routing weight (1 for the shared expert); rows past
       // the matrix (an expert's last tile) and tokens past T are zero
       float v[kDecodeN];
-      const bool valid = f.row0 + rloc < f.rows;
 #pragma unroll
       for (int c = 0; c < kDecodeN; ++c) {
         const float w = f.shared ? (c < p.T ? 1.f : 0.f) : sh.seg_w[f.slot][c];
-        const float a = __uint_as_float(r[c]) * rsc[c];
+        const float a = __uint_as_float(r[c]) * rsc[c] * srow;
         v[c] = valid && w != 0.f ? (a > 0.f ? a * a : 0.f) * w : 0.f;
       }
       // buffer b is free once unit n - 2's down MMAs have completed
@@ -1031,9 +1287,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   } else {
     // ------------------------------------------------------------- routing
     const int rt = threadIdx.x - 192;
-    route_logits<MAXT>(p, sh, rt, rl);
-    route_select(p, sh, rt, abort, kBarRoute, false);
+    route_logits<MAXT>(p, sh, rt, rl, conv);
+    const bool routed_ok = route_select(p, sh, rt, abort, kBarRoute, false);
     if (rt == 0) mbar_arrive(&sh.routed);  // (also on failure: the waiters then see abort)
+    if (conv && routed_ok && !*abort) {
+      Units ur = un;
+      ur.N = un.nS + sh.U * un.nI;
+      dequant_stages(p, sh, ur, tiles, rt, abort);
+    }
   }
 
   // ----------------------------------------------- reduction and wind down
@@ -1079,33 +1340,52 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
 
 bool fused_decode_supported(const moe_config& c, int grid) {
   // the routing warps hold a token row in kMaxChunks 8-element chunks each;
-  // the H x 16 down accumulator fits next to the two up accumulators in TMEM
-  return grid > 0 && c.latent_size == 0 && c.expert_wdtype == MOE_WEIGHTS_BF16 &&
-         c.shared_wdtype == MOE_WEIGHTS_BF16 &&
+  // the H x 16 down accumulator fits next to the two up accumulators in TMEM;
+  // FP8 routed experts (with row scales) need a BF16 shared expert, whose
+  // units then take CTAs of their own: at most half of the grid
+  const int nS = (c.shared_inter + kBM - 1) / kBM;
+  const bool experts_ok = c.expert_wdtype == MOE_WEIGHTS_BF16 ||
+                          (c.expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE && 2 * nS <= grid);
+  return grid > 0 && c.latent_size == 0 && experts_ok && c.shared_wdtype == MOE_WEIGHTS_BF16 &&
          c.hidden_size <= kMaxChunks * kRouteThreads * 8 &&
          (c.hidden_size + kBM - 1) / kBM <= kMaxRowTiles;
 }
 
+namespace {
+
+template <int MAXT, bool F8>
+cudaError_t set_smem() {
+  return cudaFuncSetAttribute(decode_fused_kernel<MAXT, F8>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kSmemOf(F8) + int(sizeof(Shared)));
+}
+
+template <bool F8>
+cudaError_t launch_bucket(const cudaLaunchConfig_t& cfg, int T, const FusedParams& p) {
+  if (T <= 1) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<1, F8>, p);
+  if (T <= 2) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<2, F8>, p);
+  if (T <= 4) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<4, F8>, p);
+  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<8, F8>, p);
+}
+
+}  // namespace
+
 cudaError_t prepare_fused_decode() {
-  const int bytes = kSmem + int(sizeof(Shared));
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(decode_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                bytes)) != cudaSuccess)
+  if ((e = set_smem<1, false>()) != cudaSuccess || (e = set_smem<2, false>()) != cudaSuccess ||
+      (e = set_smem<4, false>()) != cudaSuccess || (e = set_smem<8, false>()) != cudaSuccess ||
+      (e = set_smem<1, true>()) != cudaSuccess || (e = set_smem<2, true>()) != cudaSuccess ||
+      (e = set_smem<4, true>()) != cudaSuccess || (e = set_smem<8, true>()) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(decode_fused_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                bytes)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(decode_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                bytes)) != cudaSuccess)
-    return e;
-  return cudaFuncSetAttribute(decode_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              bytes);
+  return cudaSuccess;
 }
 
 cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   const moe_config& c = *a.cfg;
   if (!fused_decode_supported(c, a.grid) || a.T < 1 || a.T > kDecodeMaxT)
     return cudaErrorInvalidValue;
+  const bool f8 = c.expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE;
+  if (f8 && (!a.w->up_scale || !a.w->down_scale)) return cudaErrorInvalidValue;
   FusedParams p;
   p.tm_up = *a.tm_up;
   p.tm_sup = *a.tm_sup;
@@ -1119,6 +1399,8 @@ cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   p.norm_w = static_cast<const bf16*>(a.w->norm_w);
   p.gate_w = static_cast<const bf16*>(a.w->gate_w);
   p.gate_bias = a.w->gate_bias;
+  p.up_scale = f8 ? a.w->up_scale : nullptr;
+  p.down_scale = f8 ? a.w->down_scale : nullptr;
   p.T = a.T;
   p.H = c.hidden_size;
   p.E = c.num_experts;
@@ -1132,17 +1414,14 @@ cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmem + sizeof(Shared);
+  cfg.dynamicSmemBytes = kSmemOf(f8) + sizeof(Shared);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.T <= 1) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<1>, p);
-  if (a.T <= 2) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<2>, p);
-  if (a.T <= 4) return cudaLaunchKernelEx(&cfg, decode_fused_kernel<4>, p);
-  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<8>, p);
+  return f8 ? launch_bucket<true>(cfg, a.T, p) : launch_bucket<false>(cfg, a.T, p);
 }
 
 }  // namespace moe

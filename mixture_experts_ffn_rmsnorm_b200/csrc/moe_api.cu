@@ -541,6 +541,16 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
 
 // Decode path (T <= 8): one cooperative launch (decode_fused.cu) with the
 // weights as the 128-row operand and the tokens as N = 16.
+// Whether MOE_PATH_AUTO takes the decode launch.  With FP8 routed experts
+// only one token does: the launch then dequantises the weights in shared
+// memory, which pays while every routed unit has a CTA to itself (one
+// token) and not beyond (measured on B200 with the skewed FP8 workload's
+// layer: 75 against 98 us at T = 1, 118 against 104 us at T = 2).
+bool decode_preferred(const moe_handle* h, int T) {
+  return T <= MOE_DECODE_MAX_TOKENS && moe::fused_decode_supported(h->cfg, h->num_sms) &&
+         (h->cfg.expert_wdtype == MOE_WEIGHTS_BF16 || T == 1);
+}
+
 // out: where the output rows go (null: hidden, in place).
 moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cudaStream_t st,
                           moe::LaunchLog* log, bf16* out = nullptr) {
@@ -666,8 +676,7 @@ moe_status moe_forward_path(moe_handle* h, void* hidden, void* residual, int32_t
   log.nevents = h->n_stage_events;
   log.begin(s);
   const bool decode = path == MOE_PATH_DECODE ||
-                      (path == MOE_PATH_AUTO && num_tokens <= MOE_DECODE_MAX_TOKENS &&
-                       moe::fused_decode_supported(h->cfg, h->num_sms));
+                      (path == MOE_PATH_AUTO && decode_preferred(h, num_tokens));
   if (decode) {
     st = enqueue_decode(h, static_cast<bf16*>(hidden), static_cast<bf16*>(residual), num_tokens,
                         s, &log);
@@ -698,7 +707,7 @@ moe_status moe_forward_host(moe_handle* h, void* hidden_host, void* residual_hos
   // Decode sizes with page-locked buffers the device can address: the
   // kernel writes the output rows (and the residual) into them itself, so
   // no copy back and no launch of one follow the forward.
-  if (num_tokens <= MOE_DECODE_MAX_TOKENS && moe::fused_decode_supported(h->cfg, h->num_sms)) {
+  if (decode_preferred(h, num_tokens)) {
     void* out_dev = mapped_device_pointer(hidden_host);
     void* res_dev = out_dev && residual_host ? mapped_device_pointer(residual_host) : nullptr;
     if (out_dev && (!residual_host || res_dev)) {
