@@ -334,7 +334,7 @@ def config_of(s, T, path):
 # the token count its configuration names; decode also at T = 8, the largest
 # batch of the decode path.
 SUB_WORKLOADS = (("decode", 8), ("tiny", 16), ("prefill", 1024), ("latent", 4096),
-                 ("skew_fp8", 8192))
+                 ("skew_fp8", 8192), ("skew_fp8", 1))  # (the last: its FP8 layer at decode)
 
 STAGE_NOTE = ("per-kernel times come from a second CUDA graph with events recorded between "
               "the kernels; those events break the programmatic-dependent-launch overlap, so "
