@@ -153,7 +153,7 @@ def test_committed_dram_captures_are_close_to_the_model():
         name, tok = workload.split(" T=")
         T = int(tok)
         s = WORKLOADS[name]
-        path = "decode" if name == "decode" else "prefill"
+        path = "decode" if stage == "decode_fused" else "prefill"
         # touched experts: as captured (decode), all of them (prefill)
         U = rec.get("distinct_experts", s.k * T) if path == "decode" else s.E
         model = dict((m[0], m) for m in bench.stage_model(s, T, path, U, router_split=True))
