@@ -145,8 +145,12 @@ typedef enum {
 /* Validate the configuration and weights, build the TMA descriptors and
  * allocate the workspace on the current device.  Mirrors NemotronMoeLayer
  * `new` (nemotron_moe.rs): refuses top_k outside 1..=num_experts or above
- * the routing bounds.  On success *out receives a handle; on failure *out is
- * set to NULL and nothing stays allocated. */
+ * the routing bounds.  The workspace keeps a copy of the gate with the norm
+ * weight folded in (for the prefill router, which multiplies the raw rows
+ * by it), made here and synchronously: norm_w and gate_w must not change
+ * while the handle lives (the other weights are read at every forward).
+ * On success *out receives a handle; on failure *out is set to NULL and
+ * nothing stays allocated. */
 MOE_API moe_status moe_create(const moe_config* config, const moe_weights* weights, moe_handle** out);
 
 /* One forward pass over num_tokens tokens, enqueued on `stream`

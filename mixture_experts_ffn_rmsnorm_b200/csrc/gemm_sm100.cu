@@ -193,6 +193,8 @@ __device__ __forceinline__ void router_epilogue(const GemmParams& p, const GemmC
   }
   TopK tk;
   tk.init();
+  // the accumulator holds G' . x; the token's factor makes it the logits
+  const float rsc = p.topk_rs && rvalid ? p.topk_rs[row] : 1.f;
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
@@ -201,7 +203,8 @@ __device__ __forceinline__ void router_epilogue(const GemmParams& p, const GemmC
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int e = c * 32 + j;
-      if (e < E) tk.offer(e, __uint_as_float(r[j]), p.gate_bias ? p.gate_bias[e] : 0.0f, p.top_k);
+      if (e < E)
+        tk.offer(e, __uint_as_float(r[j]) * rsc, p.gate_bias ? p.gate_bias[e] : 0.0f, p.top_k);
     }
   }
   const int mt = t.row0 / kBM;
@@ -273,9 +276,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // Everything above overlaps the previous kernel when launched with PDL.
-  // Dependents may start once every CTA is past its wait, i.e. once this
-  // launch's own inputs are complete.
-  pdl_wait();
+  // Dependents may start once every CTA is past this point.  With epi_wait
+  // the producer and the MMA warp go on at once (their operands do not
+  // depend on the previous kernel) and only the epilogue warps wait; every
+  // CTA still waits before it exits, so the launch completes after the
+  // previous one.
+  if (!p.epi_wait || warp >= 2) pdl_wait();
   pdl_trigger();
 
   const int m0 = p.n_mtiles ? *p.n_mtiles : p.cls[0].mtiles;
@@ -329,8 +335,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sb = sa + Tr::kABytes;
           mbar_arrive_expect_tx(&full[stage], Tr::kStageBytes);
           const int kx = kb * bk;
+          const int kax = C.a_kwrap ? (kx % C.a_kwrap) : kx;
           const int kbx = C.b_kwrap ? (kx % C.b_kwrap) : kx;
-          tma_load_2d(sa, &p.tmA[t.c], &full[stage], kx, t.arow);
+          tma_load_2d(sa, &p.tmA[t.c], &full[stage], kax, t.arow);
           tma_load_2d(sb, &p.tmB[t.c], &full[stage], kbx, t.brow);
           ++issued;
           if (++stage == STAGES) {

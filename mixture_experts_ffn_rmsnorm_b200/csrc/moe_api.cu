@@ -108,7 +108,9 @@ struct moe_handle {
   // workspace
   void* ws;
   size_t ws_bytes;
-  bf16* gate_a;    // [Tm, 2H]: normed bf16 (hi) | residual of the rounding (lo)
+  bf16* gate_a;    // [Tm, 2H]: normed bf16 rows in the first H columns
+  bf16* gate_w2;   // [E, 2H]: the gate with the norm weight folded in, BF16 hi | lo (set at create)
+  float* rs;       // [Tm]: each token's RMSNorm factor rsqrt(mean x^2 + eps)
   int32_t* idx;    // [Tm*k]
   float* wts;      // [Tm*k]  (immediately after idx, as the pages' scratch layout)
   int32_t* off;    // [E+1]
@@ -143,7 +145,7 @@ struct moe_handle {
   float* m_scale;    // [Tm]
   moe::FusedWorkspace dec;
   // tensor maps
-  CUtensorMap tm_gate_a, tm_gate_b, tm_fc1_a, tm_fc1_b;
+  CUtensorMap tm_gate_b, tm_fc1_a, tm_fc1_b;
   CUtensorMap tm_up_a, tm_up_b, tm_sup_a, tm_sup_b;
   CUtensorMap tm_down_a, tm_down_b, tm_sdown_a, tm_sdown_b;
   // the same weights with up_bn / down_bn-row boxes (B operand of the
@@ -238,6 +240,8 @@ void carve(moe_handle* h, char* base) {
   const size_t Rm = Tm * k, D = h->D, I = c.moe_inter, S = c.shared_inter, L = c.latent_size;
   Carver cv{base};
   h->gate_a = cv.take<bf16>(Tm * 2 * H);
+  h->gate_w2 = cv.take<bf16>(size_t(E) * 2 * H);
+  h->rs = cv.take<float>(Tm);
   h->idx = cv.take<int32_t>(Rm);
   h->wts = cv.take<float>(Rm);
   h->off = cv.take<int32_t>(E + 1);
@@ -292,8 +296,7 @@ bool build_maps(moe_handle* h) {
   const uint64_t lb = lf8 ? 1 : 2;  // fc1 / fc2
   bool ok = true;
   // router: A = [hi | lo] (K = 2H), B = gate [E, H] (k wraps at H)
-  ok &= make_map(&h->tm_gate_a, h->gate_a, false, 2 * H, Tm, 2 * H * 2, moe::kBM);
-  ok &= make_map(&h->tm_gate_b, h->w.gate_w, false, H, E, H * 2, h->gate_bn);
+  ok &= make_map(&h->tm_gate_b, h->gate_w2, false, 2 * H, E, 2 * H * 2, h->gate_bn);
   if (L) {  // FP8 fc1 / fc2 read the E4M3 normed tokens / latent sums
     if (lf8)
       ok &= make_map(&h->tm_fc1_a, h->nq, true, H, Tm, H, moe::kBM);
@@ -362,12 +365,20 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
   const moe_config& c = h->cfg;
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
-  p.tmA[0] = h->tm_gate_a;
+  // The router fused with the RMSNorm (NemotronMoeLayer `prefill`: the gate
+  // runs on the normed rows): the raw rows x, read twice along K (the A
+  // coordinate wraps at H), times [G'hi | G'lo] with G' = G * norm_w; each
+  // token's logits are then r * (G' . x) = G . n, r applied in the epilogue.
+  // Only the epilogue needs the RMSNorm launch (its factors r), so the
+  // router's loads and MMAs start before that launch ends.
+  if (!make_map(&p.tmA[0], hidden, false, c.hidden_size, T, c.hidden_size * 2, moe::kBM))
+    return MOE_ERR_CUDA;
   p.tmB[0] = h->tm_gate_b;
   p.cls[0] = dense_class(2 * c.hidden_size, c.num_experts, T, moe::EPI_TOPK, nullptr, 0,
                          h->gate_bn);
   p.cls[0].ntiles = 1;
-  p.cls[0].b_kwrap = c.hidden_size;
+  p.cls[0].a_kwrap = c.hidden_size;
+  p.topk_rs = h->rs;
   p.nclasses = 1;
   if (with_fc1 && c.latent_size > 0) {
     p.tmA[1] = h->tm_fc1_a;
@@ -402,8 +413,10 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
     ks = (nk + per - 1) / per;  // every split non-empty
   }
   p.cls[0].ksplit = ks;
+  // (fc1's operand is the normed rows: with it in the launch every warp waits)
+  p.epi_wait = p.nclasses == 1;
   MOE_TRY(moe::launch_rmsnorm(hidden, static_cast<const bf16*>(h->w.norm_w), residual, h->gate_a,
-                              h->need_nq && with_fc1 ? h->nq : nullptr, h->nq_scale, T,
+                              h->rs, h->need_nq && with_fc1 ? h->nq : nullptr, h->nq_scale, T,
                               c.hidden_size, c.rms_eps, ks > 1 ? h->expert_hist : nullptr,
                               mt * c.num_experts, st));
   log->done(st);
@@ -419,12 +432,12 @@ moe_status enqueue_route(moe_handle* h, const bf16* hidden, bf16* residual, int 
   p.status = h->status;
   int W = mt * ks + (p.nclasses > 1 ? p.cls[1].mtiles * p.cls[1].ntiles : 0);
   const int grid = W < h->num_sms ? W : h->num_sms;
-  MOE_TRY(moe::launch_grouped_gemm(p, h->gate_bn, grid, st));
+  MOE_TRY(moe::launch_grouped_gemm(p, h->gate_bn, grid, st, /*pdl=*/true));
   log->done(st);
   if (ks > 1) {
     MOE_TRY(moe::launch_router_reduce(h->topk_part, ks, mt * moe::kBM, T, c.num_experts,
-                                      h->w.gate_bias, c.top_k, c.routed_scaling_factor, h->idx,
-                                      h->wts, h->expert_hist, st));
+                                      h->w.gate_bias, c.top_k, c.routed_scaling_factor, h->rs,
+                                      h->idx, h->wts, h->expert_hist, st));
     log->done(st);
   }
   return MOE_OK;
@@ -635,7 +648,11 @@ moe_status moe_create(const moe_config* config, const moe_weights* weights, moe_
   h->ws = ws;
   carve(h, static_cast<char*>(ws));
   if (cudaMemset(ws, 0, h->ws_bytes) != cudaSuccess || !build_maps(h) ||
-      moe::prepare_grouped_gemm() != cudaSuccess || moe::prepare_fused_decode() != cudaSuccess) {
+      moe::prepare_grouped_gemm() != cudaSuccess || moe::prepare_fused_decode() != cudaSuccess ||
+      moe::launch_prep_gate(static_cast<const bf16*>(h->w.gate_w),
+                            static_cast<const bf16*>(h->w.norm_w), config->num_experts,
+                            config->hidden_size, h->gate_w2, 0) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(ws);
     h->magic = 0;
     delete h;

@@ -58,6 +58,7 @@ struct GemmClass {
   int ntiles;             // ceil(N / BN)
   int mtiles;             // m-tiles of a dense class (ignored when the launch has a tile table)
   int rows;               // valid A rows of a dense class
+  int a_kwrap;            // A's k coordinate is taken modulo this (0 = no wrap)
   int b_kwrap;            // B's k coordinate is taken modulo this (0 = no wrap)
   int ksplit;             // dense classes: K-block ranges per output tile (0 or 1 = whole K)
   int epi;                // EpiKind
@@ -87,6 +88,7 @@ struct GemmParams {
   float rsf;
   int* topk_idx;
   float* topk_w;
+  const float* topk_rs;    // per-row factor of the logits (the token's RMSNorm factor) or null
   float* topk_part;        // split-K partial logits [ksplit][topk_rows_cap][E]
   int topk_rows_cap;
   int* expert_hist;        // [token tiles][E] experts chosen by each 128-token tile
@@ -94,6 +96,10 @@ struct GemmParams {
   const float* blend_s;
   const __nv_bfloat16* blend_res;
   int* status;
+  // Only the epilogue warps wait for the previous launch (griddepcontrol):
+  // the operands the producer loads do not depend on it, only what the
+  // epilogue reads does (the router: the RMSNorm factors).
+  int epi_wait;
   // Dynamic tile schedule (null = static round-robin):
   // sched[0] hands out tile indices past the first gridDim.x, sched[1]
   // counts exiting CTAs.  Both are zero before the launch and the last CTA
@@ -113,21 +119,27 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, int bn, int grid, cudaStrea
 cudaError_t prepare_grouped_gemm();
 
 // Routing / sort / data movement kernels (route.cu).
+// RMSNorm: residual <- hidden, rs[t] = rsqrt(mean x^2 + eps), bf16 normed
+// rows into the first H columns of gate_a [T, 2H].
 // normed_q/normed_scale (nullable): per-token E4M3 copy of the normed rows.
 // hist_clear[0..n_clear) is zeroed on the way (the split-K router's
 // histogram, accumulated with atomics); may be null.
 cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* norm_w,
-                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, uint8_t* normed_q,
-                           float* normed_scale, int T, int H, float eps, int* hist_clear,
-                           int n_clear, cudaStream_t stream);
-// Split-K router, second half: logits = sum of the ks partials in split
-// order, sigmoid top-k per token into idx/w, and hist[t / 128][e] += 1 for
-// every chosen expert (hist zeroed beforehand).  Launched as a programmatic
-// dependent of the router GEMM.
+                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, float* rs,
+                           uint8_t* normed_q, float* normed_scale, int T, int H, float eps,
+                           int* hist_clear, int n_clear, cudaStream_t stream);
+// The router's gate with the norm weight folded in: out [E, 2H] =
+// [bf16(G * w) | bf16(G * w - bf16(G * w))] (fp32 products), once per layer.
+cudaError_t launch_prep_gate(const __nv_bfloat16* gate, const __nv_bfloat16* norm_w, int E, int H,
+                             __nv_bfloat16* out, cudaStream_t stream);
+// Split-K router, second half: logits = rs[t] * the sum of the ks partials
+// in split order, sigmoid top-k per token into idx/w, and hist[t / 128][e]
+// += 1 for every chosen expert (hist zeroed beforehand).  Launched as a
+// programmatic dependent of the router GEMM.
 constexpr int kRouterMaxSplit = 16;
 cudaError_t launch_router_reduce(const float* part, int ks, int rows_cap, int T, int E,
-                                 const float* bias, int k, float rsf, int* idx, float* w,
-                                 int* hist, cudaStream_t stream);
+                                 const float* bias, int k, float rsf, const float* rs, int* idx,
+                                 float* w, int* hist, cudaStream_t stream);
 // Stable sort by expert from the routing table idx [T, k] and its per-128-
 // token-tile expert histogram hist [ceil(T/128), E].
 cudaError_t launch_tile_hist(const int* idx, int T, int k, int E, int* hist, int* status,

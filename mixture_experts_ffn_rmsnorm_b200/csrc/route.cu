@@ -64,17 +64,20 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 
 // RMSNorm of one token per block (NemotronMoeLayer `prefill`: rms_norm_residual
 // writes the normed activations and the residual).  residual <- hidden; the
-// normed vector n = x * rsqrt(mean(x^2) + eps) * w is written as two BF16
-// halves into gate_a [T, 2H]: hi = bf16(n) (this is also the experts' input)
-// and lo = bf16(n - hi), so the router GEMM on [hi | lo] x [G | G] sees n to
-// about 16 significant bits (FP32-accurate logits from BF16 tensor cores).
-// With FP8 experts it also writes an E4M3 copy of n with one float scale per
-// token (scale = max|n| / 448).  hist_clear[0..n_clear) is zeroed.
+// factor r = rsqrt(mean(x^2) + eps) goes to rs[t], and the normed vector
+// n = x * r * w, rounded to BF16, to the first H columns of gate_a [T, 2H]
+// (the experts', the shared expert's and fc1's input).  The router does not
+// read n: it multiplies the raw x by the gate with w folded in and applies r
+// to its logits (prep_gate_kernel).  With FP8 experts it also writes an E4M3
+// copy of n with one float scale per token (scale = max|n| / 448).
+// hist_clear[0..n_clear) is zeroed.  The next launch (the router, whose main
+// loop reads only x and the gate) may start at once.
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ norm_w,
     __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ gate_a,
-    uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale, int H, float eps,
-    int* __restrict__ hist_clear, int n_clear) {
+    float* __restrict__ rs, uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale,
+    int H, float eps, int* __restrict__ hist_clear, int n_clear) {
+  pdl_trigger();
   __shared__ float red[kNormThreads / 32];
   const int t = blockIdx.x;
   for (int i = t * kNormThreads + threadIdx.x; i < n_clear; i += gridDim.x * kNormThreads)
@@ -92,23 +95,20 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(
     for (int j = 0; j < 8; ++j) ss += f[j] * f[j];
   }
   const float r = rsqrtf(block_reduce(ss, red, false) / float(H) + eps);
+  if (threadIdx.x == 0) rs[t] = r;
   const uint4* w = reinterpret_cast<const uint4*>(norm_w);
   uint4* hi = reinterpret_cast<uint4*>(gate_a + size_t(t) * 2 * H);
-  uint4* lo = hi + nv;
   float amax = 0.f;
   for (int i = threadIdx.x; i < nv; i += kNormThreads) {
-    float f[8], g[8], h[8], l[8];
+    float f[8], g[8], h[8];
     unpack8(x[i], f);
     unpack8(w[i], g);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float n = f[j] * r * g[j];
-      h[j] = __bfloat162float(__float2bfloat16_rn(n));
-      l[j] = n - h[j];
-      amax = fmaxf(amax, fabsf(n));
+      h[j] = f[j] * r * g[j];
+      amax = fmaxf(amax, fabsf(h[j]));
     }
     hi[i] = pack8(h);
-    lo[i] = pack8(l);
   }
   if (!normed_q) return;
   amax = block_reduce(amax, red, true);
@@ -134,8 +134,9 @@ template <int MAXC>
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ norm_w,
     __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ gate_a,
-    uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale, int H, float eps,
-    int* __restrict__ hist_clear, int n_clear) {
+    float* __restrict__ rs, uint8_t* __restrict__ normed_q, float* __restrict__ normed_scale,
+    int H, float eps, int* __restrict__ hist_clear, int n_clear) {
+  pdl_trigger();
   __shared__ float red[kNormThreads / 32];
   const int t = blockIdx.x;
   for (int i = t * kNormThreads + threadIdx.x; i < n_clear; i += gridDim.x * kNormThreads)
@@ -166,25 +167,22 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(
     }
   }
   const float r = rsqrtf(block_reduce(ss, red, false) / float(H) + eps);
+  if (threadIdx.x == 0) rs[t] = r;
   uint4* hi = reinterpret_cast<uint4*>(gate_a + size_t(t) * 2 * H);
-  uint4* lo = hi + nv;
   float amax = 0.f;
 #pragma unroll
   for (int c = 0; c < MAXC; ++c) {
     const int i = threadIdx.x + c * kNormThreads;
     if (i < nv) {
-      float f[8], g[8], h[8], l[8];
+      float f[8], g[8], h[8];
       unpack8(xv[c], f);
       unpack8(wv[c], g);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float n = f[j] * r * g[j];
-        h[j] = __bfloat162float(__float2bfloat16_rn(n));
-        l[j] = n - h[j];
-        amax = fmaxf(amax, fabsf(n));
+        h[j] = f[j] * r * g[j];
+        amax = fmaxf(amax, fabsf(h[j]));
       }
       hi[i] = pack8(h);
-      lo[i] = pack8(l);
     }
   }
   if (!normed_q) return;
@@ -207,6 +205,26 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(
   }
 }
 
+// The router's gate with the norm weight folded in, as two BF16 halves
+// (once, when the layer is created): g'[e, i] = G[e, i] * w[i] in fp32,
+// out[e] = [bf16(g') | bf16(g' - bf16(g'))] [E, 2H].  The router multiplies
+// the token rows x (BF16, exact) by both halves, so that it sums
+// x_i * g'_ei to about 16 significant bits per term: with r applied to the
+// sum, logit = r * (G . (x * w)) = G . n in float32 accuracy.
+__global__ void prep_gate_kernel(const __nv_bfloat16* __restrict__ gate,
+                                 const __nv_bfloat16* __restrict__ norm_w, int E, int H,
+                                 __nv_bfloat16* __restrict__ out) {
+  const size_t n = size_t(E) * H;
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n;
+       i += size_t(gridDim.x) * blockDim.x) {
+    const size_t e = i / H, c = i - e * H;
+    const float g = __bfloat162float(gate[i]) * __bfloat162float(norm_w[c]);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(g);
+    out[e * 2 * H + c] = hi;
+    out[e * 2 * H + H + c] = __float2bfloat16_rn(g - __bfloat162float(hi));
+  }
+}
+
 // Split-K router, second half (one warp per token).  Lane l sums the
 // partial logits of experts l, l + 32, ... over the splits in split order
 // (two splits' loads in flight at a time, each warp load one coalesced
@@ -214,8 +232,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(
 // and adds the token's choices to its 128-token tile's expert histogram.
 __global__ void __launch_bounds__(256) router_reduce_kernel(
     const float* __restrict__ part, int ks, int rows_cap, int T, int E,
-    const float* __restrict__ bias, int k, float rsf, int* __restrict__ idx,
-    float* __restrict__ w, int* __restrict__ hist) {
+    const float* __restrict__ bias, int k, float rsf, const float* __restrict__ rs,
+    int* __restrict__ idx, float* __restrict__ w, int* __restrict__ hist) {
   pdl_wait();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -243,6 +261,10 @@ __global__ void __launch_bounds__(256) router_reduce_kernel(
     for (int j = 0; j < 8; ++j)
       acc[j] += j < nj && lane + 32 * j < E ? __ldcg(src + size_t(s) * sstride + 32 * j) : 0.f;
   }
+  // the partials are G' . x: the token's factor r makes them the logits
+  const float r = rs[t];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] *= r;
   const int e = warp_topk_regs(acc, bias, E, k, rsf, idx + size_t(t) * k, w + size_t(t) * k);
   // (an out-of-range id comes only from NaN logits; the sort flags it)
   if (lane < k && unsigned(e) < unsigned(E)) atomicAdd(hist + size_t(t / kBM) * E + e, 1);
@@ -551,28 +573,35 @@ __global__ void latent_reduce_kernel(const __nv_bfloat16* __restrict__ y,
 }  // namespace
 
 cudaError_t launch_rmsnorm(const __nv_bfloat16* hidden, const __nv_bfloat16* norm_w,
-                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, uint8_t* normed_q,
-                           float* normed_scale, int T, int H, float eps, int* hist_clear,
-                           int n_clear, cudaStream_t stream) {
+                           __nv_bfloat16* residual, __nv_bfloat16* gate_a, float* rs,
+                           uint8_t* normed_q, float* normed_scale, int T, int H, float eps,
+                           int* hist_clear, int n_clear, cudaStream_t stream) {
   const int nc = hist_clear ? n_clear : 0;
   const int chunks = (H / 8 + kNormThreads - 1) / kNormThreads;
   if (chunks <= 2)
-    rmsnorm_reg_kernel<2><<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a,
+    rmsnorm_reg_kernel<2><<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, rs,
                                                           normed_q, normed_scale, H, eps,
                                                           hist_clear, nc);
   else if (chunks <= 8)
-    rmsnorm_reg_kernel<8><<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a,
+    rmsnorm_reg_kernel<8><<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, rs,
                                                           normed_q, normed_scale, H, eps,
                                                           hist_clear, nc);
   else
-    rmsnorm_kernel<<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, normed_q,
-                                                   normed_scale, H, eps, hist_clear, nc);
+    rmsnorm_kernel<<<T, kNormThreads, 0, stream>>>(hidden, norm_w, residual, gate_a, rs,
+                                                   normed_q, normed_scale, H, eps, hist_clear,
+                                                   nc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_gate(const __nv_bfloat16* gate, const __nv_bfloat16* norm_w, int E, int H,
+                             __nv_bfloat16* out, cudaStream_t stream) {
+  prep_gate_kernel<<<592, 256, 0, stream>>>(gate, norm_w, E, H, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_router_reduce(const float* part, int ks, int rows_cap, int T, int E,
-                                 const float* bias, int k, float rsf, int* idx, float* w,
-                                 int* hist, cudaStream_t stream) {
+                                 const float* bias, int k, float rsf, const float* rs, int* idx,
+                                 float* w, int* hist, cudaStream_t stream) {
   if (ks < 2 || ks > kRouterMaxSplit || E > 256) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((T + 7) / 8);
@@ -584,7 +613,7 @@ cudaError_t launch_router_reduce(const float* part, int ks, int rows_cap, int T,
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, router_reduce_kernel, part, ks, rows_cap, T, E, bias, k, rsf,
-                            idx, w, hist);
+                            rs, idx, w, hist);
 }
 
 cudaError_t launch_quantize_rows(const __nv_bfloat16* u, unsigned* u_amax, uint8_t* uq,
