@@ -82,16 +82,20 @@ def stage_model(s, T, path, U, router_split=False):
         # in L2 and are not counted)
         nb, fl, f8f = step_work(s, T, U)
         return [("decode_fused", nb, fl, f8f)]
-    st = [("rmsnorm", T * H * 2 * 2 + T * 2 * H * 2 + (T * H if s.expert_fp8 else 0), 0, 0)]
+    # RMSNorm: x in, residual and the bf16 normed rows out, r per token (and
+    # the E4M3 copy with FP8 experts)
+    st = [("rmsnorm", T * H * 2 * 3 + T * 4 + (T * H + T * 4 if s.expert_fp8 else 0), 0, 0)]
     # With split K (few token tiles) the router GEMM stores partial logits
     # and a second kernel sums them and selects; its algorithmic bytes are
     # the routing table it writes (the partials are the split's overhead).
     sel = "" if router_split else "_topk"
+    # the router reads the raw rows x (once; its second pass along K hits L2)
+    # and the gate with the norm weight folded in, as BF16 hi and lo halves
     if L:
-        st.append((f"router_gemm{sel}+fc1", E * H * 2 + T * 2 * H * 2 + L * H * 2 + T * L * 2,
-                   2 * T * E * H + 2 * T * H * L, 0))
+        st.append((f"router_gemm{sel}+fc1", E * 2 * H * 2 + T * H * 2 + L * H * 2 + T * H * 2
+                   + T * L * 2, 2 * T * E * H + 2 * T * H * L, 0))
     else:
-        st.append((f"router_gemm{sel}", E * H * 2 + T * 2 * H * 2 + (0 if router_split else R * 8),
+        st.append((f"router_gemm{sel}", E * 2 * H * 2 + T * H * 2 + (0 if router_split else R * 8),
                    2 * T * E * H, 0))
     if router_split:
         st.append(("router_reduce_topk", R * 8, 0, 0))
