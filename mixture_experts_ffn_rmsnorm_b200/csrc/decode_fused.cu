@@ -213,6 +213,7 @@ struct Shared {
   int stop;                 // the epilogue warps' common decision to stop (epi_stop)
   int route_fail;
   int conv_stop;            // the dequantising warps' common decision to stop
+  int has_partial;          // the epilogue warps staged this CTA's partial output
   int flag;
   int U;                    // routed slots
   float rs[kDecodeMaxT];
@@ -227,6 +228,8 @@ struct Shared {
 };
 
 static_assert(kSmemOf(false) + sizeof(Shared) <= 227 * 1024, "shared memory of one CTA");
+static_assert(kDecodeMaxT * kMaxChunks * kRouteThreads * 8 * 4 <= kStages * kStageBytes,
+              "a CTA's partial output [T, H] fp32 is staged in the idle ring");
 static_assert(kSmemOf(true) + sizeof(Shared) <= 227 * 1024, "shared memory of one CTA (FP8)");
 static_assert(kStagesF8 <= kStages, "barrier arrays");
 
@@ -323,7 +326,7 @@ __device__ __forceinline__ bool step_of(const Units& u, int m, int s, int* kind,
 template <int MAXT>
 struct RouteLoads {
   static constexpr bool kHold = MAXT <= 2;
-  static constexpr int kHeld = kHold ? kMaxChunks : 1;
+  static constexpr int kHeld = kHold ? kMaxChunks : 2;  // (more tokens: two chunks at a time)
   uint4 x[kHeld][MAXT], w[kHeld], a[kHeld], b[kHeld];
 };
 
@@ -411,10 +414,13 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoad
 #pragma unroll
     for (int j = 0; j < kMaxChunks; ++j) consume(j, L.x[j], L.w[j], L.a[j], L.b[j]);
   } else {
+    // two chunks' loads in flight at a time
 #pragma unroll 1
-    for (int j = 0; j < kMaxChunks; ++j) {
+    for (int j = 0; j < kMaxChunks; j += 2) {
       route_load_chunk<MAXT>(p, rt, j, L.x[0], L.w[0], L.a[0], L.b[0]);
+      route_load_chunk<MAXT>(p, rt, j + 1, L.x[1], L.w[1], L.a[1], L.b[1]);
       consume(j, L.x[0], L.w[0], L.a[0], L.b[0]);
+      consume(j + 1, L.x[1], L.w[1], L.a[1], L.b[1]);
     }
   }
   if (rt < E) sh.bias[rt] = p.gate_bias ? p.gate_bias[rt] : 0.f;
@@ -810,6 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   uint8_t* ubufs = tiles + kRingBytes(F8);  // two relu^2 row buffers
   Shared& sh = *reinterpret_cast<Shared*>(ubufs + 2 * kUBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr bool kStagePartial = MAXT >= 4;
   const int G = gridDim.x, cta = blockIdx.x;
   const int nH = (p.H + kBM - 1) / kBM;
   const int kbH = p.H / 64;
@@ -854,6 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     }
     sh.abort = 0;
     sh.U = 0;
+    sh.has_partial = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -1262,12 +1270,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       if (tid == 0) mbar_arrive(&sh.ufull[b]);
     }
     // this CTA's partial output (the H x 16 down accumulator, columns < T)
-    // into the launch's fixed-point sum
+    // into the launch's fixed-point sum.  From four tokens on, the partial
+    // goes to shared memory, token-major [T, H] (the ring is idle once every
+    // down MMA has completed), and all warps issue the T x H adds below (at
+    // T = 8 this shortens the tail by about 1 us); below four, the epilogue
+    // warps add it themselves (the extra barrier would cost more)
     if (ok && m > 0) {
       if (lane == 0 && !mbar_wait(&sh.down_done, 0, abort)) record_timeout(p.status, abort);
       __syncwarp();
       if (!epi_stop(sh, tid)) {
         tc_fence_after();
+        float* stagef = reinterpret_cast<float*>(tiles);
         for (int rt = 0; rt < nH; ++rt) {
           uint32_t r[16];
           tmem_ld_32x32b_x16(lane_base + uint32_t((2 + rt) * kDecodeN), r);
@@ -1275,13 +1288,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           const int row = rt * kBM + rloc;
           if (row < p.H) {
 #pragma unroll
-            for (int c = 0; c < MAXT; ++c)
-              if (c < p.T) add_partial(p.ws, size_t(c) * p.H + row, __uint_as_float(r[c]));
+            for (int c = 0; c < MAXT; ++c) {
+              if (c >= p.T) continue;
+              if constexpr (kStagePartial)
+                stagef[c * p.H + row] = __uint_as_float(r[c]);
+              else
+                add_partial(p.ws, size_t(c) * p.H + row, __uint_as_float(r[c]));
+            }
           }
         }
         tc_fence_before();
         named_barrier(kBarEpi, kEpiThreads);
-        if (tid == 0) red_release_add(p.ws.sync + kPartialsDone, 1u);
+        if (tid == 0) {
+          if constexpr (kStagePartial)
+            sh.has_partial = 1;
+          else
+            red_release_add(p.ws.sync + kPartialsDone, 1u);
+        }
       }
     }
   } else {
@@ -1303,6 +1326,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+  // this CTA's partial output, staged by the epilogue warps, into the
+  // launch's fixed-point sum: every warp issues the T x H atomic adds
+  if (kStagePartial && sh.has_partial) {
+    const float* stagef = reinterpret_cast<const float*>(tiles);
+    const int n = p.T * p.H;
+    for (int i = threadIdx.x; i < n; i += kThreads) add_partial(p.ws, size_t(i), stagef[i]);
+    __syncthreads();
+    if (threadIdx.x == 0) red_release_add(p.ws.sync + kPartialsDone, 1u);
   }
   // Rows [r0, r0 + nr) of the output, once every CTA that had units has
   // added its partial and every CTA's logits are in (after that no CTA reads

@@ -508,8 +508,22 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, const int* _
     const float4 a = s4[0], b = s4[1];
     acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
     acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-    for (int j = 0; j < k; ++j) {
-      unpack8(reinterpret_cast<const uint4*>(y + size_t(rows[j]) * H)[i], f);
+    // two rows' loads in flight per step (the same order of additions)
+    int j = 0;
+    for (; j + 2 <= k; j += 2) {
+      const uint4 ya = __ldcs(reinterpret_cast<const uint4*>(y + size_t(rows[j]) * H) + i);
+      const uint4 yb = __ldcs(reinterpret_cast<const uint4*>(y + size_t(rows[j + 1]) * H) + i);
+      float fb[8];
+      unpack8(ya, f);
+      unpack8(yb, fb);
+      const float wa = wts[j], wb = wts[j + 1];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += wa * f[q];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += wb * fb[q];
+    }
+    if (j < k) {
+      unpack8(__ldcs(reinterpret_cast<const uint4*>(y + size_t(rows[j]) * H) + i), f);
       const float wj = wts[j];
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] += wj * f[q];
@@ -538,8 +552,22 @@ __global__ void latent_reduce_kernel(const __nv_bfloat16* __restrict__ y,
   float amax = 0.f;
   for (int i = threadIdx.x; i < nv; i += blockDim.x) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, f[8];
-    for (int j = 0; j < k; ++j) {
-      unpack8(reinterpret_cast<const uint4*>(y + size_t(rows[j]) * L)[i], f);
+    // two rows' loads in flight per step (the same order of additions)
+    int j = 0;
+    for (; j + 2 <= k; j += 2) {
+      const uint4 ya = __ldcs(reinterpret_cast<const uint4*>(y + size_t(rows[j]) * L) + i);
+      const uint4 yb = __ldcs(reinterpret_cast<const uint4*>(y + size_t(rows[j + 1]) * L) + i);
+      float fb[8];
+      unpack8(ya, f);
+      unpack8(yb, fb);
+      const float wa = wts[j], wb = wts[j + 1];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += wa * f[q];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += wb * fb[q];
+    }
+    if (j < k) {
+      unpack8(__ldcs(reinterpret_cast<const uint4*>(y + size_t(rows[j]) * L) + i), f);
       const float wj = wts[j];
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] += wj * f[q];
