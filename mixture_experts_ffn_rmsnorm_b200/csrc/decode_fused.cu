@@ -214,6 +214,7 @@ struct Shared {
   int route_fail;
   int conv_stop;            // the dequantising warps' common decision to stop
   int has_partial;          // the epilogue warps staged this CTA's partial output
+  uint32_t partial_tokens;  // its token columns that are not exactly zero
   int flag;
   int U;                    // routed slots
   float rs[kDecodeMaxT];
@@ -245,7 +246,10 @@ __device__ __forceinline__ bool epi_stop(Shared& sh, int tid) {
 
 // ------------------------------------------------------------------ units
 // Units: shared-expert tiles j < nS, then routed tile (j - nS) % nI of slot
-// (j - nS) / nI.  CTA c takes j = c, c + grid, c + 2 grid, ...  With FP8
+// (j - nS) / nI.  CTA c takes j = c, c + grid, c + 2 grid, ...  (Neighbouring
+// CTAs thus stream neighbouring tiles of an expert at the same time; its
+// down slices share DRAM rows.  Giving each CTA a contiguous run of routed
+// tiles instead made the T = 8 stream about 8 us slower.)  With FP8
 // routed experts the two kinds stay on separate CTAs (a CTA's stages are
 // either BF16 or FP8): CTA c < nS takes shared unit c alone, and the routed
 // units go round-robin over the other Gr = grid - nS CTAs.  Its steps:
@@ -316,19 +320,29 @@ __device__ __forceinline__ bool step_of(const Units& u, int m, int s, int* kind,
 // loads; the epilogue applies r_t to accumulator column t instead
 // (W . (x r w) = r (W . (x w))).
 //
-// One or two tokens: every chunk's loads are in flight at once, issued
-// first of all, before the launch's set-up (route_issue): the routing
-// decides when the routed weights can stream, and the set-up's cold
-// instruction fetches then overlap the loads' DRAM latency (2.5 us earlier
-// routing at T = 1).  More tokens would spill those registers: their chunks
-// go one at a time, in route_logits (issuing the first one early was
-// slower at T = 8).
+// One or two tokens: every routing thread takes chunks rt, rt + 128, ...
+// of every token, and all their loads are in flight at once, issued first
+// of all, before the launch's set-up (route_issue): the routing decides
+// when the routed weights can stream, and the set-up's cold instruction
+// fetches then overlap the loads' DRAM latency (2.5 us earlier routing at
+// T = 1).
+//
+// Three or four tokens: the same mapping, two chunks' loads in flight at a
+// time.  Five to eight tokens: routing warp w owns tokens w and w + 4, and
+// its lanes stride over the chunks, kTokChunks of them in flight
+// (route_tokwarp).  Unrolled over eight tokens, the first mapping's loop
+// body is large, and its first pass (cold instruction cache after the L2
+// flush) took about 3.5 us per chunk; the token rows are then ready 2.8 us
+// later at T = 8 (at T = 4 the warp-per-token loop, with three rounds of
+// loads instead of two, is 0.5 us slower).
 template <int MAXT>
 struct RouteLoads {
   static constexpr bool kHold = MAXT <= 2;
-  static constexpr int kHeld = kHold ? kMaxChunks : 2;  // (more tokens: two chunks at a time)
+  static constexpr bool kTokWarp = MAXT > 4;
+  static constexpr int kHeld = kHold ? kMaxChunks : 2;  // (3-4 tokens: two chunks at a time)
   uint4 x[kHeld][MAXT], w[kHeld], a[kHeld], b[kHeld];
 };
+constexpr int kTokChunks = 4;  // chunks in flight per lane with a warp per token
 
 // Chunk j of routing thread rt: the norm weight, this CTA's gate rows and
 // the tokens, 8 elements each.
@@ -359,11 +373,114 @@ __device__ __forceinline__ void route_issue(const FusedParams& p, int rt, RouteL
   }
 }
 
-// f16tok: write the token rows as f16 instead of BF16 (the up GEMM of FP8
-// units runs on f16 operands).
+// Five to eight tokens (see RouteLoads): warp w of the routing warps sums
+// tokens w and w + 4 over all of H, lane l taking chunks l, l + 32, ...,
+// kTokChunks at a time.  The norm weight and this CTA's gate rows are loaded
+// by every warp (L2 hits after the first).  Same products as route_hold;
+// each token's sums are reduced within its warp.
 template <int MAXT>
-__device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoads<MAXT>& L,
-                             bool f16tok) {
+__device__ __forceinline__ void route_tokwarp(const FusedParams& p, Shared& sh, int rt,
+                                              bool f16tok) {
+  constexpr int TPW = (MAXT + 3) / 4;  // tokens per warp
+  const int H = p.H, T = p.T, E = p.E, G = gridDim.x;
+  const int nv = H / 8;
+  const int warp = rt >> 5, lane = rt & 31;
+  const int e0 = blockIdx.x, e1 = blockIdx.x + G;
+  const bool has0 = e0 < E, has1 = e1 < E;
+  bf16* x16 = p.ws.x16 + size_t(blockIdx.x) * kDecodeN * H;
+  float ss[TPW], d0[TPW], d1[TPW];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) ss[i] = d0[i] = d1[i] = 0.f;
+  if (warp < T) {
+#pragma unroll 1
+    for (int c0 = lane; c0 < nv; c0 += 32 * kTokChunks) {
+      uint4 xq[kTokChunks][TPW], wq[kTokChunks], aq[kTokChunks], bq[kTokChunks];
+#pragma unroll
+      for (int u = 0; u < kTokChunks; ++u) {
+        const int c = c0 + 32 * u;
+        const bool in = c < nv;
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        wq[u] = in ? __ldg(reinterpret_cast<const uint4*>(p.norm_w) + c) : z;
+        aq[u] = in && has0 ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e0) * H) + c)
+                           : z;
+        bq[u] = in && has1 ? __ldcs(reinterpret_cast<const uint4*>(p.gate_w + size_t(e1) * H) + c)
+                           : z;
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          const int t = warp + 4 * i;
+          xq[u][i] = in && t < T ? reinterpret_cast<const uint4*>(p.hidden + size_t(t) * H)[c] : z;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kTokChunks; ++u) {
+        const int c = c0 + 32 * u;
+        float w[8], a[8], b[8];
+        unpack8(wq[u], w);
+        unpack8(aq[u], a);
+        unpack8(bq[u], b);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          a[q] *= w[q];
+          b[q] *= w[q];
+        }
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          const int t = warp + 4 * i;
+          float f[8];
+          unpack8(xq[u][i], f);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            ss[i] += f[q] * f[q];
+            d0[i] += a[q] * f[q];
+            d1[i] += b[q] * f[q];
+          }
+          if (c < nv && t < T) {
+            reinterpret_cast<uint4*>(x16 + size_t(t) * H)[c] =
+                f16tok ? make_uint4(pack_f16x2(f[0] * w[0], f[1] * w[1]),
+                                    pack_f16x2(f[2] * w[2], f[3] * w[3]),
+                                    pack_f16x2(f[4] * w[4], f[5] * w[5]),
+                                    pack_f16x2(f[6] * w[6], f[7] * w[7]))
+                       : make_uint4(pack_bf16x2(f[0] * w[0], f[1] * w[1]),
+                                    pack_bf16x2(f[2] * w[2], f[3] * w[3]),
+                                    pack_bf16x2(f[4] * w[4], f[5] * w[5]),
+                                    pack_bf16x2(f[6] * w[6], f[7] * w[7]));
+            if (blockIdx.x == 0) reinterpret_cast<uint4*>(p.residual + size_t(t) * H)[c] = xq[u][i];
+          }
+        }
+      }
+    }
+  }
+  if (rt < E) sh.bias[rt] = p.gate_bias ? p.gate_bias[rt] : 0.f;
+  if (rt + kRouteThreads < E)
+    sh.bias[rt + kRouteThreads] = p.gate_bias ? p.gate_bias[rt + kRouteThreads] : 0.f;
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    const int t = warp + 4 * i;
+    const float v0 = warp_sum(ss[i]), v1 = warp_sum(d0[i]), v2 = warp_sum(d1[i]);
+    if (lane == 0 && t < T) {
+      const float r = rsqrtf(v0 / float(H) + p.eps);
+      sh.rs[t] = r;
+      if (has0) p.ws.logits[t * E + e0] = v1 * r;
+      if (has1) p.ws.logits[t * E + e1] = v2 * r;
+    }
+  }
+  // the token rows: generic writes -> the TMA loads of this CTA's producer
+  fence_proxy_async_global();
+  named_barrier(kBarRoute, kRouteThreads);
+  // the token rows, their factors r_t and every logit of this CTA are in
+  // place (and, CTA 0, the residual): the weight stream may start
+  if (rt == 0) {
+    mbar_arrive(&sh.loads_out);
+    mbar_arrive(&sh.tokens);
+    red_release_add(p.ws.sync + kRouteArrived, 1u);
+  }
+}
+
+// One to four tokens (see RouteLoads); with one or two, from the loads
+// route_issue made.
+template <int MAXT>
+__device__ void route_hold(const FusedParams& p, Shared& sh, int rt, RouteLoads<MAXT>& L,
+                           bool f16tok) {
   const int H = p.H, T = p.T, E = p.E, G = gridDim.x;
   const int nv = H / 8;
   const int warp = rt >> 5, lane = rt & 31;
@@ -461,6 +578,18 @@ __device__ void route_logits(const FusedParams& p, Shared& sh, int rt, RouteLoad
     mbar_arrive(&sh.tokens);
     red_release_add(p.ws.sync + kRouteArrived, 1u);
   }
+}
+
+// The routing pass of the routing warps (see RouteLoads).  f16tok: write the
+// token rows as f16 instead of BF16 (the up GEMM of FP8 units runs on f16
+// operands).
+template <int MAXT>
+__device__ __forceinline__ void route_logits(const FusedParams& p, Shared& sh, int rt,
+                                             RouteLoads<MAXT>& L, bool f16tok) {
+  if constexpr (RouteLoads<MAXT>::kTokWarp)
+    route_tokwarp<MAXT>(p, sh, rt, f16tok);
+  else
+    route_hold<MAXT>(p, sh, rt, L, f16tok);
 }
 
 // The sigmoid top-k of token t by one warp, into sel_idx / sel_w.  The dry
@@ -1207,6 +1336,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
     bool ok = true, routed = false;
     int m = un.shared_first() ? 1 : 0;
+    // the tokens this CTA's units reach: its partial output is exactly zero
+    // in every other column (their relu^2 rows are zero), which it need not add
+    uint32_t tmask = 0;
     for (int n = 0; ok; ++n) {
       if (n >= m) {
         if (routed) break;
@@ -1225,6 +1357,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       const UnitInfo f = unit_info(p, sh, un, n);
       const int b = n & 1;
       const uint32_t par = (n >> 1) & 1;
+#pragma unroll
+      for (int c = 0; c < MAXT; ++c)
+        if (c < p.T && (f.shared || sh.seg_w[f.slot][c] != 0.f)) tmask |= 1u << c;
       const bool valid = f.row0 + rloc < f.rows;
       // an FP8 unit's up runs on the unscaled E4M3 values: its row's scale
       // (loaded while the up runs)
@@ -1289,7 +1424,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           if (row < p.H) {
 #pragma unroll
             for (int c = 0; c < MAXT; ++c) {
-              if (c >= p.T) continue;
+              if (!((tmask >> c) & 1u)) continue;
               if constexpr (kStagePartial)
                 stagef[c * p.H + row] = __uint_as_float(r[c]);
               else
@@ -1300,9 +1435,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         tc_fence_before();
         named_barrier(kBarEpi, kEpiThreads);
         if (tid == 0) {
-          if constexpr (kStagePartial)
+          if constexpr (kStagePartial) {
+            sh.partial_tokens = tmask;
             sh.has_partial = 1;
-          else
+          } else
             red_release_add(p.ws.sync + kPartialsDone, 1u);
         }
       }
@@ -1331,8 +1467,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   // launch's fixed-point sum: every warp issues the T x H atomic adds
   if (kStagePartial && sh.has_partial) {
     const float* stagef = reinterpret_cast<const float*>(tiles);
-    const int n = p.T * p.H;
-    for (int i = threadIdx.x; i < n; i += kThreads) add_partial(p.ws, size_t(i), stagef[i]);
+    const uint32_t tm = sh.partial_tokens;
+    for (int c = 0; c < p.T; ++c) {
+      if (!((tm >> c) & 1u)) continue;
+      for (int i = threadIdx.x; i < p.H; i += kThreads)
+        add_partial(p.ws, size_t(c) * p.H + i, stagef[c * p.H + i]);
+    }
     __syncthreads();
     if (threadIdx.x == 0) red_release_add(p.ws.sync + kPartialsDone, 1u);
   }
