@@ -203,7 +203,9 @@ MOE_API moe_status moe_route(moe_handle* h, const void* hidden, int32_t num_toke
 /* Sort-by-expert of given routing idx [T, k] (device): perm [R] (sorted
  * position -> flat row t*k + j), inv [R] (flat row -> sorted position), off
  * [E+1] (exclusive prefix of per-expert counts).  Rows of one expert keep
- * token order.  Device pointers; idx values must lie in [0, E). */
+ * token order.  Device pointers; idx values must lie in [0, E): a row with
+ * an id outside it is left out of perm and off, gets inv = -1, and sets bit 2
+ * of the device status word (moe_get_device_status). */
 MOE_API moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_tokens, int32_t* perm,
                     int32_t* inv, int32_t* off, void* stream);
 
@@ -228,9 +230,9 @@ MOE_API moe_status moe_sort(moe_handle* h, const int32_t* idx, int32_t num_token
  *   status: optional device int32; set to 0, then bit 2 is OR-ed in if an
  *   id lies outside [0, num_experts) (that row is skipped).  NULL uses a
  *   word in the scratch that the caller cannot read: a bad id then goes
- *   unreported, and the entries of perm and inv it would have filled
- *   (perm[off[E]..R) and inv of its row) are left unwritten.  Pass a status
- *   word unless the ids are known to be in range.
+ *   unreported.  Either way the row gets inv = -1, and the entries of perm
+ *   it would have filled (perm[off[E]..R)) are left unwritten.  Pass a
+ *   status word unless the ids are known to be in range.
  *   stream: cudaStream_t (NULL = legacy default stream).
  *
  * Errors (nothing is launched): MOE_ERR_NULL_POINTER for a NULL idx, perm,

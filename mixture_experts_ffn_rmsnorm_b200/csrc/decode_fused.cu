@@ -1416,7 +1416,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       if (!epi_stop(sh, tid)) {
         tc_fence_after();
         float* stagef = reinterpret_cast<float*>(tiles);
-        for (int rt = 0; rt < nH; ++rt) {
+        // (below four tokens, where the CTAs finish at about the same time,
+        // each starts at its own row tile rather than all adding to the
+        // same addresses together)
+        for (int i = 0; i < nH; ++i) {
+          const int rt = kStagePartial ? i : (i + cta) % nH;
           uint32_t r[16];
           tmem_ld_32x32b_x16(lane_base + uint32_t((2 + rt) * kDecodeN), r);
           tmem_ld_wait();

@@ -449,8 +449,11 @@ __global__ void __launch_bounds__(kSortThreads) sort_tiles_kernel(
         perm[pos] = f;
         inv[f] = pos;
       } else {
+        inv[f] = -1;
         atomicOr(status, kStatusBadIndex);  // inconsistent histogram: skip the write
       }
+    } else if (f < g1) {
+      inv[f] = -1;  // an id outside [0, E) (only from NaN logits): the row goes nowhere
     }
     __syncwarp();
     if (e >= 0 && rank == 0) wh[warp][e] += __popc(peers);
@@ -485,20 +488,35 @@ __global__ void gather_kernel(const uint8_t* __restrict__ X, size_t ldx,
   if (scale && lane == 0) xs_scale[p] = scale[t];
 }
 
+// Token t's slot j (thread j < k): its sorted row and weight into rows /
+// wts.  A slot whose expert id was out of range (only from non-finite
+// logits; the sort then sets its inv to -1 and reports it) reads row 0,
+// inside the buffer, with weight 0 (it adds 0 unless that row holds a
+// non-finite value, which only the outputs of such a token may then show).
+// The loop over the slots stays branch-free.
+__device__ __forceinline__ void load_slot(const int* __restrict__ inv, const float* __restrict__ w,
+                                          int t, int k, int R, int* rows, float* wts) {
+  const int j = threadIdx.x;
+  if (j < k) {
+    const int r = inv[t * k + j];
+    const float wv = w[t * k + j];  // (both loads in flight at once)
+    const bool ok = r >= 0 && r < R;
+    rows[j] = ok ? r : 0;
+    wts[j] = ok ? wv : 0.f;
+  }
+}
+
 // hidden[t] = bf16(residual[t] + s[t] + sum_j w[t,j] * y[inv[t*k + j]])
 // (MoeLayer `forward_prefill`: unpermute + weighted reduce, shared expert
 // blend; nemotron_moe.rs module documentation: summed and added to hidden).
 __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ inv,
                                const float* __restrict__ w, const float* __restrict__ s,
                                const __nv_bfloat16* __restrict__ residual,
-                               __nv_bfloat16* __restrict__ hidden, int k, int H) {
+                               __nv_bfloat16* __restrict__ hidden, int k, int H, int R) {
   const int t = blockIdx.x;
   __shared__ int rows[kMaxTopKShared];
   __shared__ float wts[kMaxTopKShared];
-  if (threadIdx.x < k) {
-    rows[threadIdx.x] = inv[t * k + threadIdx.x];
-    wts[threadIdx.x] = w[t * k + threadIdx.x];
-  }
+  load_slot(inv, w, t, k, R, rows, wts);
   __syncthreads();
   const int nv = H / 8;
   for (int i = threadIdx.x; i < nv; i += blockDim.x) {
@@ -538,15 +556,12 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, const int* _
 __global__ void latent_reduce_kernel(const __nv_bfloat16* __restrict__ y,
                                      const int* __restrict__ inv, const float* __restrict__ w,
                                      __nv_bfloat16* __restrict__ m, uint8_t* __restrict__ mq,
-                                     float* __restrict__ m_scale, int k, int L) {
+                                     float* __restrict__ m_scale, int k, int L, int R) {
   const int t = blockIdx.x;
   __shared__ int rows[kMaxTopKShared];
   __shared__ float wts[kMaxTopKShared];
   __shared__ float red[32];
-  if (threadIdx.x < k) {
-    rows[threadIdx.x] = inv[t * k + threadIdx.x];
-    wts[threadIdx.x] = w[t * k + threadIdx.x];
-  }
+  load_slot(inv, w, t, k, R, rows, wts);
   __syncthreads();
   const int nv = L / 8;
   float amax = 0.f;
@@ -681,14 +696,14 @@ cudaError_t launch_gather(const void* X, size_t ldx_bytes, const int* perm, int 
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* inv, const float* w, const float* s,
                            const __nv_bfloat16* residual, __nv_bfloat16* hidden, int T, int k,
                            int H, cudaStream_t stream) {
-  combine_kernel<<<T, 128, 0, stream>>>(y, inv, w, s, residual, hidden, k, H);
+  combine_kernel<<<T, 128, 0, stream>>>(y, inv, w, s, residual, hidden, k, H, T * k);
   return cudaGetLastError();
 }
 
 cudaError_t launch_latent_reduce(const __nv_bfloat16* y, const int* inv, const float* w,
                                  __nv_bfloat16* m, uint8_t* mq, float* m_scale, int T, int k,
                                  int L, cudaStream_t stream) {
-  latent_reduce_kernel<<<T, 128, 0, stream>>>(y, inv, w, m, mq, m_scale, k, L);
+  latent_reduce_kernel<<<T, 128, 0, stream>>>(y, inv, w, m, mq, m_scale, k, L, T * k);
   return cudaGetLastError();
 }
 

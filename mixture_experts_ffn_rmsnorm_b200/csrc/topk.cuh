@@ -66,48 +66,57 @@ struct TopK {
   }
 };
 
+// Order-preserving bits of a selection key: for keys a, b that are not NaN,
+// a > b exactly when key_bits(a) > key_bits(b) as unsigned integers (-0 is
+// taken as +0).  NaN maps to 0, below every other key (a NaN key is never
+// chosen: no comparison with it is true); -inf maps to kKeyNegInf.
+constexpr uint32_t kKeyNegInf = 0x007FFFFFu;
+__device__ __forceinline__ uint32_t key_bits(float f) {
+  if (f != f) return 0u;
+  const uint32_t u = __float_as_uint(f + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Warp-cooperative top-k of one token's E <= 256 logits (same selection rule
 // and weight formula as TopK): lane l holds the logits of experts l, l + 32,
-// ... in lg[]; k rounds of a warp arg-max on (key descending, expert index
-// ascending).  idx[0..k) and w[0..k) are written by the warp (global or
-// shared memory).  Returns, on lanes < k, the expert chosen in round `lane`
-// (-1 elsewhere).
+// ... in lg[].  k rounds of a warp arg-max on (key descending, expert index
+// ascending): a warp-wide integer max of the key bits, then a warp-wide min
+// of the expert indices that hold that key.  A round in which no remaining
+// key beats -inf (only with NaN or infinite inputs) chooses id 0x7fffffff,
+// as a plain scan from -inf would.  idx[0..k) and w[0..k) are written by the
+// warp (global or shared memory).  Returns, on lanes < k, the expert chosen
+// in round `lane` (-1 elsewhere).
 __device__ __forceinline__ int warp_topk_regs(const float (&lg)[8], const float* bias, int E,
                                               int k, float rsf, int* idx, float* w) {
   const int lane = threadIdx.x & 31;
-  float key[8], sc[8];
+  uint32_t key[8];
+  float sc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = lane + 32 * j;
     if (e < E) {
       const float s = 1.0f / (1.0f + expf(-lg[j]));
       sc[j] = s;
-      key[j] = s + (bias ? bias[e] : 0.0f);
+      key[j] = key_bits(s + (bias ? bias[e] : 0.0f));
     } else {
       sc[j] = 0.f;
-      key[j] = -INFINITY;
+      key[j] = kKeyNegInf;
     }
   }
   float sum = 0.f, mine = 0.f;
   int mine_e = -1;
   for (int r = 0; r < k; ++r) {
-    float bk = -INFINITY;
+    uint32_t lm = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) lm = key[j] > lm ? key[j] : lm;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
     int be = 0x7fffffff;
+    if (m > kKeyNegInf) {
+      int mi = 0x7fffffff;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (key[j] > bk) {
-        bk = key[j];
-        be = lane + 32 * j;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ok > bk || (ok == bk && oe < be)) {
-        bk = ok;
-        be = oe;
-      }
+      for (int j = 7; j >= 0; --j)
+        if (key[j] == m) mi = lane + 32 * j;
+      be = __reduce_min_sync(0xffffffffu, mi);
     }
     float s = 0.f;
     if ((be & 31) == lane) {
@@ -115,7 +124,7 @@ __device__ __forceinline__ int warp_topk_regs(const float (&lg)[8], const float*
       for (int j = 0; j < 8; ++j) {
         if (lane + 32 * j == be) {
           s = sc[j];
-          key[j] = -INFINITY;
+          key[j] = 0u;
         }
       }
     }

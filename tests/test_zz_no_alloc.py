@@ -98,6 +98,11 @@ def test_static_sort_status_is_cleared_between_calls():
     moe.sort_static(torch.from_numpy(bad).cuda(), k, E, perm, inv, off, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) & BAD_INDEX_BIT
+    # the skipped row goes nowhere (inv = -1); every other row is placed
+    inv_b, perm_b = inv.cpu().numpy(), perm.cpu().numpy()
+    assert inv_b[7 * k + 1] == -1
+    good = np.array([f for f in range(T * k) if f != 7 * k + 1])
+    assert np.array_equal(perm_b[inv_b[good]], good)
     moe.sort_static(torch.from_numpy(idx).cuda(), k, E, perm, inv, off, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
