@@ -53,6 +53,7 @@ struct FusedDecodeArgs {
   const moe_weights* w;
   const FusedWorkspace* ws;
   const CUtensorMap *tm_up, *tm_sup, *tm_down, *tm_sdown;  // weights as 128-row A boxes
+  const CUtensorMap *tm_up64, *tm_sup64;  // up weights as 64-row A boxes (units of 64 rows)
   const CUtensorMap* tm_x[4];  // token rows, B boxes of 1, 2, 4, 8 rows (token-count bucket)
   __nv_bfloat16* hidden;    // [T, H] input rows
   __nv_bfloat16* residual;  // [T, H] written with the input rows (device or mapped host memory)

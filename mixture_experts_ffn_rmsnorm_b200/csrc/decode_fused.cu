@@ -6,20 +6,23 @@
 // cooperative grid of one CTA per SM.
 //
 // The work is cut along the experts' intermediate dimension.  A unit is 128
-// intermediate rows of one expert (the shared expert's, or a routed slot's):
+// intermediate rows of a routed slot's expert (64 for its last tile when the
+// expert's size is an odd multiple of 64), or 64 rows of the shared expert:
 //   up     u = relu^2(W_up[rows] . n) (x routing weight), 128 x 16 tokens,
-//          K = H: tcgen05.mma M = 128 (weight rows), N = 16 (tokens), BF16 in,
-//          fp32 accumulate in TMEM;
-//   down   y += W_down[:, rows] . u over all H output rows (K = 128), the
+//          K = H: tcgen05.mma M = 128 (weight rows; a 64-row unit loads
+//          64-row boxes and leaves the other accumulator rows unused),
+//          N = 16 (tokens), BF16 in, fp32 accumulate in TMEM;
+//   down   y += W_down[:, rows] . u over all H output rows (K = 128 or 64), the
 //          relu^2 rows going from TMEM through shared memory as the MMA's
 //          token operand.
 // A unit needs nothing from other CTAs once the tokens are routed, and every
 // unit's down adds into the same H x 16 accumulator, which stays in TMEM
 // (ceil(H / 128) x 16 columns) until the CTA's last unit.  Unit j goes to
 // CTA j % grid: shared-expert units first (they need no routing and start at
-// once), routed units after.  At the end every CTA stores its partial H x T
-// block, and each CTA adds up one slice of rows over all CTAs' partials, in
-// CTA order (deterministic), plus the residual, into hidden.
+// once), routed units after.  At the end every CTA adds its partial H x T
+// block into an int64 fixed-point accumulator (integer addition: exact and
+// independent of the order, so the result is deterministic), and each CTA
+// finishes one slice of rows, the sum plus the residual, into hidden.
 //
 // Warp roles (320 threads):
 //   warp 0     TMA producer: weight boxes (and the up GEMM's token rows) into
@@ -56,6 +59,10 @@ using bf16 = __nv_bfloat16;
 // flight (measured with a standalone streaming probe on B200: 59 against
 // 46 GB/s per SM with 90 SMs streaming).
 constexpr int kKB = 2;
+// Rows of a shared-expert unit.  Half the routed units' 128: twice as many
+// CTAs stream the shared expert while the routing runs (its weights need no
+// routing), 58 instead of 29 at shared_inter 3712.
+constexpr int kSharedUnit = 64;
 constexpr int kStages = 5;
 constexpr int kABytes = kBM * 128;          // 128 weight rows x 64 BF16
 constexpr int kBBytes = kDecodeN * 128;     // 16 token rows x 64 BF16
@@ -112,6 +119,8 @@ struct FusedParams {
   CUtensorMap tm_sup;    // shared up weights   [S, H]
   CUtensorMap tm_down;   // routed down weights [E*H, I]
   CUtensorMap tm_sdown;  // shared down weights [H, S]
+  CUtensorMap tm_up64;   // routed up weights, 64-row boxes (an expert's last 64-row tile)
+  CUtensorMap tm_sup64;  // shared up weights, 64-row boxes (shared units are 64 rows)
   CUtensorMap tm_x;      // x16 [grid * 16, H]: 16 rows per CTA   (B, boxes of MAXT rows)
   const bf16* hidden;
   bf16* residual;
@@ -728,7 +737,8 @@ __device__ __forceinline__ void store_u_row(uint8_t* ubuf, int rloc, const float
 // (j - nS) / nI.
 struct UnitInfo {
   bool shared;
-  int slot, expert, row0, rows;  // rows: valid intermediate rows of the weight matrix (S or I)
+  int slot, expert, row0;
+  int row_end;  // first intermediate row past the unit (64 or 128 rows after row0, or S / I)
 };
 
 __device__ __forceinline__ UnitInfo unit_info(const FusedParams& p, const Shared& sh,
@@ -739,21 +749,21 @@ __device__ __forceinline__ UnitInfo unit_info(const FusedParams& p, const Shared
   if (f.shared) {
     f.slot = -1;
     f.expert = 0;
-    f.row0 = j * kBM;
-    f.rows = p.S;
+    f.row0 = j * kSharedUnit;
+    f.row_end = min(p.S, f.row0 + kSharedUnit);
   } else {
     const int r = j - u.nS;
     f.slot = r / u.nI;
     f.expert = sh.seg_expert[f.slot];
     f.row0 = (r - f.slot * u.nI) * kBM;
-    f.rows = p.I;
+    f.row_end = min(p.I, f.row0 + kBM);
   }
   return f;
 }
 
-// 64-wide k-blocks of a unit's down slice that hold weights (the last tile
-// of an expert may have only 64 valid rows).
-__device__ __forceinline__ int down_kk(const UnitInfo& f) { return f.rows - f.row0 >= kBM ? 2 : 1; }
+// 64-wide k-blocks of a unit's down slice (64 or 128 rows: S and I are
+// multiples of 64).
+__device__ __forceinline__ int down_kk(const UnitInfo& f) { return f.row_end - f.row0 > 64 ? 2 : 1; }
 
 // ------------------------------------------------------ FP8 dequantisation
 // Row r of FP8 staging slot f8 (128 rows x 128 E4M3, 128-byte swizzle: the
@@ -904,7 +914,7 @@ __device__ bool dequant_stages(const FusedParams& p, Shared& sh, const Units& un
       bool valid;
       float scale;
       if (kind == 0) {
-        valid = f.row0 + rt < f.rows;
+        valid = f.row0 + rt < f.row_end;
         scale = 1.f;
       } else {
         valid = i * kBM + rt < p.H;
@@ -953,7 +963,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   Units un;
   un.c = cta;
   un.G = G;
-  un.nS = (p.S + kBM - 1) / kBM;
+  un.nS = (p.S + kSharedUnit - 1) / kSharedUnit;
   un.nI = (p.I + kBM - 1) / kBM;
   un.N = un.nS;  // the routed units are added once the routing is known
   un.f8 = F8;
@@ -998,6 +1008,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     tma_prefetch_desc(&p.tm_sup);
     tma_prefetch_desc(&p.tm_down);
     tma_prefetch_desc(&p.tm_sdown);
+    tma_prefetch_desc(&p.tm_up64);
+    tma_prefetch_desc(&p.tm_sup64);
     tma_prefetch_desc(&p.tm_x);
   }
   if (warp == 1) {
@@ -1048,7 +1060,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       }
       // nk <= kKB consecutive k-blocks into the next free stage: weight boxes
       // at x = ax, ax + 64, ... (and for up the token boxes at bx, bx + 64, ...)
-      auto issue = [&](const CUtensorMap* map, int ax, int ay, int nk, bool up, int bx) -> bool {
+      auto issue = [&](const CUtensorMap* map, int ax, int ay, int nk, bool up, int bx,
+                       uint32_t abytes) -> bool {
         if (!mbar_test_wait(&sh.empty[stage], phase ^ 1u)) {
           const long long t0 = clock64();
           // try_wait suspends this thread (no issue slots taken from the
@@ -1069,7 +1082,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         uint8_t* sa = tiles + stage * kStageBytes;
         // (a token box holds MAXT rows: the MMA reads all 16 rows of the slot,
         // but rows past T only reach accumulator columns the epilogue drops)
-        mbar_arrive_expect_tx(&sh.full[stage], uint32_t(nk * (up ? kABytes + MAXT * 128 : kABytes)));
+        mbar_arrive_expect_tx(&sh.full[stage], uint32_t(nk * (up ? abytes + MAXT * 128 : abytes)));
         for (int i = 0; i < nk; ++i)
           tma_load_2d_hint(sa + i * kABytes, map, &sh.full[stage], ax + i * 64, ay, stream_policy);
         if (up) {
@@ -1161,15 +1174,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
               ok = issue8(&p.tm_down, f.row0, f.expert * p.H + r * kBM, false, 0);
           }
         } else if (kind == 0) {  // up: W_up[rows] x tokens, K = H
-          const CUtensorMap* map = f.shared ? &p.tm_sup : &p.tm_up;
+          // (a unit of 64 rows loads 64-row boxes: the stage's other 64
+          // A rows keep stale data, whose accumulator rows are not used)
+          const bool half = f.row_end - f.row0 <= 64;
+          const CUtensorMap* map = f.shared ? (half ? &p.tm_sup64 : &p.tm_sup)
+                                            : (half ? &p.tm_up64 : &p.tm_up);
           const int ay = f.shared ? f.row0 : f.expert * p.I + f.row0;
+          const uint32_t ab = half ? uint32_t(kABytes / 2) : uint32_t(kABytes);
           for (int kb = 0; ok && kb < kbH; kb += kKB)
-            ok = issue(map, kb * 64, ay, min(kKB, kbH - kb), true, kb * 64);
+            ok = issue(map, kb * 64, ay, min(kKB, kbH - kb), true, kb * 64, ab);
         } else {  // down: W_down[:, rows] for every 128-row block of H
           const CUtensorMap* map = f.shared ? &p.tm_sdown : &p.tm_down;
           const int nkk = down_kk(f);
           for (int r = 0; ok && r < nH; ++r)
-            ok = issue(map, f.row0, (f.shared ? 0 : f.expert * p.H) + r * kBM, nkk, false, 0);
+            ok = issue(map, f.row0, (f.shared ? 0 : f.expert * p.H) + r * kBM, nkk, false, 0,
+                       uint32_t(kABytes));
         }
       }
       // the remaining token loads (also on an abort, so that every issued
@@ -1360,7 +1379,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
 #pragma unroll
       for (int c = 0; c < MAXT; ++c)
         if (c < p.T && (f.shared || sh.seg_w[f.slot][c] != 0.f)) tmask |= 1u << c;
-      const bool valid = f.row0 + rloc < f.rows;
+      const bool valid = f.row0 + rloc < f.row_end;
       // an FP8 unit's up runs on the unscaled E4M3 values: its row's scale
       // (loaded while the up runs)
       const float srow = conv && !f.shared && valid
@@ -1519,7 +1538,7 @@ bool fused_decode_supported(const moe_config& c, int grid) {
   // the H x 16 down accumulator fits next to the two up accumulators in TMEM;
   // FP8 routed experts (with row scales) need a BF16 shared expert, whose
   // units then take CTAs of their own: at most half of the grid
-  const int nS = (c.shared_inter + kBM - 1) / kBM;
+  const int nS = (c.shared_inter + kSharedUnit - 1) / kSharedUnit;
   const bool experts_ok = c.expert_wdtype == MOE_WEIGHTS_BF16 ||
                           (c.expert_wdtype == MOE_WEIGHTS_FP8_E4M3_ROWSCALE && 2 * nS <= grid);
   return grid > 0 && c.latent_size == 0 && experts_ok && c.shared_wdtype == MOE_WEIGHTS_BF16 &&
@@ -1567,6 +1586,8 @@ cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   p.tm_sup = *a.tm_sup;
   p.tm_down = *a.tm_down;
   p.tm_sdown = *a.tm_sdown;
+  p.tm_up64 = *a.tm_up64;
+  p.tm_sup64 = *a.tm_sup64;
   const int bucket = a.T <= 1 ? 0 : a.T <= 2 ? 1 : a.T <= 4 ? 2 : 3;
   p.tm_x = *a.tm_x[bucket];
   p.hidden = a.hidden;

@@ -151,6 +151,8 @@ struct moe_handle {
   // the same weights with up_bn / down_bn-row boxes (B operand of the
   // prefill launches; the decode launches read them as the 128-row A operand)
   CUtensorMap tm_up_w, tm_sup_w, tm_down_w, tm_sdown_w;
+  // the up weights with 64-row boxes (the decode launch's units of 64 rows)
+  CUtensorMap tm_up_b64, tm_sup_b64;
   int up_bn, down_bn;
   CUtensorMap tm_fc2_a, tm_fc2_b;
   CUtensorMap tm_dec_x[4];  // decode token rows, one 16-row block per CTA; boxes of 1, 2, 4, 8 rows
@@ -315,6 +317,8 @@ bool build_maps(moe_handle* h) {
   else
     ok &= make_map(&h->tm_sup_a, h->gate_a, false, H, Tm, 2 * H * 2, moe::kBM);
   ok &= make_map(&h->tm_sup_b, h->w.shared_up_w, sf8, H, S, H * sb, 128);
+  ok &= make_map(&h->tm_up_b64, h->w.up_w, f8, D, E * I, D * eb, 64);
+  ok &= make_map(&h->tm_sup_b64, h->w.shared_up_w, sf8, H, S, H * sb, 64);
   // grouped down: routed A = u [Rm, I], B = down [E*D, I]; shared A = v, B = [H, S]
   ok &= make_map(&h->tm_down_a, f8 ? static_cast<const void*>(h->uq) : h->u, f8, I, Rm, I * eb,
                  moe::kBM);
@@ -578,6 +582,8 @@ moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cu
   a.tm_sup = &h->tm_sup_b;    // shared up weights [S, H]
   a.tm_down = &h->tm_down_b;  // routed down weights [E*H, I]
   a.tm_sdown = &h->tm_sdown_b;
+  a.tm_up64 = &h->tm_up_b64;  // the same up weights, 64-row boxes
+  a.tm_sup64 = &h->tm_sup_b64;
   for (int b = 0; b < 4; ++b) a.tm_x[b] = &h->tm_dec_x[b];
   a.hidden = hidden;
   a.residual = residual;
