@@ -221,7 +221,6 @@ struct Shared {
   int abort;
   int stop;                 // the epilogue warps' common decision to stop (epi_stop)
   int route_fail;
-  int conv_stop;            // the dequantising warps' common decision to stop
   int has_partial;          // the epilogue warps staged this CTA's partial output
   uint32_t partial_tokens;  // its token columns that are not exactly zero
   int flag;
@@ -895,17 +894,17 @@ __device__ bool dequant_stages(const FusedParams& p, Shared& sh, const Units& un
     }
 #pragma unroll 1
     for (int i = 0; i < nstage; ++i) {
-      // one thread waits (bounded) for the slot's data and the stage's
-      // room, then all take its decision together (no thread may leave a
-      // named barrier's count short)
-      if (rt == 0) {
-        const bool ok = mbar_wait(&sh.f8full[fs], fph, abort) &&
-                        mbar_wait(&sh.empty[st], sph ^ 1u, abort);
+      // Each warp on its own (no named barrier between the four): lane 0
+      // waits (bounded) for the slot's data and the stage's room, the warp
+      // takes its decision, converts its 32 rows and counts itself in on
+      // the stage and the slot (four arrivals each).
+      const int lane = rt & 31;
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(&sh.f8full[fs], fph, abort) && mbar_wait(&sh.empty[st], sph ^ 1u, abort);
         if (!ok) record_timeout(p.status, abort);
-        sh.conv_stop = !ok;
       }
-      named_barrier(kBarRoute, kRouteThreads);
-      if (sh.conv_stop) return false;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
       // (both phases are complete: every thread observes them itself)
       mbar_wait(&sh.f8full[fs], fph, abort);
       mbar_wait(&sh.empty[st], sph ^ 1u, abort);
@@ -928,8 +927,8 @@ __device__ bool dequant_stages(const FusedParams& p, Shared& sh, const Units& un
       else
         dequant_row<false>(slots + fs * kF8SlotBytes, tiles + st * kStageBytes, rt, scale, valid);
       fence_proxy_async_shared();  // generic writes -> tensor core reads
-      named_barrier(kBarRoute, kRouteThreads);
-      if (rt == 0) {
+      __syncwarp();
+      if (lane == 0) {
         mbar_arrive(&sh.full[st]);
         mbar_arrive(&sh.f8empty[fs]);
       }
@@ -976,8 +975,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   if (warp >= 6) route_issue<MAXT>(p, threadIdx.x - 192, rl);
 
   if (threadIdx.x == 0) {
+    // (a dequantising CTA's stages are filled by the four routing warps)
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.full[s], conv ? kRouteThreads / 32 : 1);
       mbar_init(&sh.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -995,7 +995,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     if (F8) {
       for (int s = 0; s < kF8Slots; ++s) {
         mbar_init(&sh.f8full[s], 1);
-        mbar_init(&sh.f8empty[s], 1);
+        mbar_init(&sh.f8empty[s], kRouteThreads / 32);  // freed by the four routing warps
       }
     }
     sh.abort = 0;
