@@ -372,6 +372,9 @@ def measure(inp, T, args, world, flush, peaks, *, e2e=True):
 
     import mixture_experts_ffn_rmsnorm_b200 as moe
 
+    fpath = {"auto": moe.PATH_AUTO, "decode": moe.PATH_DECODE,
+             "prefill": moe.PATH_PREFILL}[getattr(args, "path", "auto")]
+
     shape = inp.shape
     layer = moe.MoELayer.from_inputs(inp, max_tokens=T)
     hbits = inp.hidden[:T]
@@ -382,7 +385,7 @@ def measure(inp, T, args, world, flush, peaks, *, e2e=True):
 
     # one untimed step to learn the launch count, the path and the routing
     hid.copy_(pristine)
-    layer.forward(hid, res)
+    layer.forward(hid, res, path=fpath)
     torch.cuda.synchronize()
     nl = layer.last_launch_count()
     path = "decode" if layer.last_path_decode() else "prefill"
@@ -400,7 +403,7 @@ def measure(inp, T, args, world, flush, peaks, *, e2e=True):
     for _ in range(args.warmup):
         flush()
         hid.copy_(pristine)
-        layer.forward(hid, res)
+        layer.forward(hid, res, path=fpath)
     torch.cuda.synchronize()
 
     # The step: one replay of a CUDA graph of the forward (what a serving loop
@@ -413,11 +416,11 @@ def measure(inp, T, args, world, flush, peaks, *, e2e=True):
         side.wait_stream(stream)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side):
-            layer.forward(hid, res, stream=side)
+            layer.forward(hid, res, path=fpath, stream=side)
         prof_graph = torch.cuda.CUDAGraph()
         layer.set_stage_events(prof_events)
         with torch.cuda.graph(prof_graph, stream=side):
-            layer.forward(hid, res, stream=side)
+            layer.forward(hid, res, path=fpath, stream=side)
         layer.set_stage_events(None)
         stream.wait_stream(side)
         for _ in range(args.warmup):
@@ -440,7 +443,7 @@ def measure(inp, T, args, world, flush, peaks, *, e2e=True):
             if graph is not None:
                 graph.replay()
             else:
-                layer.forward(hid, res)
+                layer.forward(hid, res, path=fpath)
             e_end[i].record(stream)
         torch.cuda.synchronize()
         if world > 1:
@@ -462,13 +465,15 @@ def measure(inp, T, args, world, flush, peaks, *, e2e=True):
         if prof_graph is not None:
             prof_graph.replay()
         else:
-            layer.forward(hid, res)
+            layer.forward(hid, res, path=fpath)
         torch.cuda.synchronize()
         stage_ms[i] = [prof_events[j].elapsed_time(prof_events[j + 1]) for j in range(nl)]
     layer.set_stage_events(None)
 
     e2e_rec = None
-    if e2e:
+    # (the host-buffer entry point chooses the path itself: no end-to-end
+    # figure for a forced path)
+    if e2e and getattr(args, "path", "auto") == "auto":
         # end to end through the host-buffer entry point (pinned host memory)
         h_host = torch.from_numpy(hbits.view(np.int16).copy()).pin_memory()
         e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -526,6 +531,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--path", default="auto", choices=["auto", "decode", "prefill"],
+                    help="force the decode launch or the prefill path (default: the "
+                         "library's own choice); a forced path reports no e2e figure")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
@@ -572,7 +580,10 @@ def main():
                     cache.clear()
                     cache[name] = make_inputs(WORKLOADS[name], T=Ts)
                 sub_inp = cache[name]
-            r = measure(sub_inp, Ts, args, world, flush, peaks)
+            # (the workload records take the library's own path choice)
+            r = measure(sub_inp, Ts, dataclasses.replace(args, path="auto")
+                        if dataclasses.is_dataclass(args) else
+                        argparse.Namespace(**{**vars(args), "path": "auto"}), world, flush, peaks)
             subs.append({"workload": config_of(WORKLOADS[name], Ts, r["path"])["workload"],
                          "tokens_per_step": Ts, "metric": METRIC, "unit": UNIT,
                          "dtype": "fp8+bf16" if WORKLOADS[name].expert_fp8 else "bf16",
