@@ -27,6 +27,7 @@ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 // resets the synchronisation words.
 struct FusedWorkspace {
   __nv_bfloat16* x16;      // [CTAs, 16, H] each CTA's copy of bf16(n) of the tokens (rows >= T unused)
+  uint8_t* x8;             // [CTAs, 16, H] E4M3 copy of x * w (one-token FP8 launch, W8A8; row 0 used)
   float* logits;           // [8, E]
   int* idx;                // [8, k] routing of the pass (for moe_copy_routing)
   float* w;                // [8, k]
@@ -40,6 +41,7 @@ template <class Take>
 void carve_fused(FusedWorkspace* d, const moe_config& c, int ctas, Take take) {
   const size_t k = c.top_k, E = c.num_experts, H = c.hidden_size;
   d->x16 = reinterpret_cast<__nv_bfloat16*>(take(size_t(ctas) * kDecodeN * H * 2));
+  d->x8 = reinterpret_cast<uint8_t*>(take(size_t(ctas) * kDecodeN * H));
   d->logits = reinterpret_cast<float*>(take(kDecodeMaxT * E * 4));
   d->idx = reinterpret_cast<int*>(take(kDecodeMaxT * k * 4));
   d->w = reinterpret_cast<float*>(take(kDecodeMaxT * k * 4));
@@ -55,6 +57,7 @@ struct FusedDecodeArgs {
   const CUtensorMap *tm_up, *tm_sup, *tm_down, *tm_sdown;  // weights as 128-row A boxes
   const CUtensorMap *tm_up64, *tm_sup64;  // up weights as 64-row A boxes (units of 64 rows)
   const CUtensorMap* tm_x[4];  // token rows, B boxes of 1, 2, 4, 8 rows (token-count bucket)
+  const CUtensorMap* tm_x8;    // E4M3 token rows (x8), boxes of one row x 128 bytes
   __nv_bfloat16* hidden;    // [T, H] input rows
   __nv_bfloat16* residual;  // [T, H] written with the input rows (device or mapped host memory)
   __nv_bfloat16* out;       // [T, H] output rows (device or mapped host memory); null: hidden

@@ -63,6 +63,13 @@ constexpr int kKB = 2;
 // CTAs stream the shared expert while the routing runs (its weights need no
 // routing), 58 instead of 29 at shared_inter 3712.
 constexpr int kSharedUnit = 64;
+// W8A8 at one token (FusedParams::w8): the token chooses top_k distinct
+// experts, and when their routed units fit on the CTAs beside the shared
+// expert's, every such CTA has one unit, whose accumulators hold one
+// expert's products alone.  The MMA then reads the E4M3 weight boxes from
+// the staging slots as they land (kind::f8f6f4), with the token row and the
+// relu^2 rows in E4M3 (one scale each, amax / 448), and the epilogues apply
+// the weight row scales and those two scales: no dequantisation at all.
 constexpr int kStages = 5;
 constexpr int kABytes = kBM * 128;          // 128 weight rows x 64 BF16
 constexpr int kBBytes = kDecodeN * 128;     // 16 token rows x 64 BF16
@@ -121,6 +128,7 @@ struct FusedParams {
   CUtensorMap tm_sdown;  // shared down weights [H, S]
   CUtensorMap tm_up64;   // routed up weights, 64-row boxes (an expert's last 64-row tile)
   CUtensorMap tm_sup64;  // shared up weights, 64-row boxes (shared units are 64 rows)
+  CUtensorMap tm_x8;     // x8 [grid * 16, H] E4M3 token rows (W8A8 launch), one-row boxes
   CUtensorMap tm_x;      // x16 [grid * 16, H]: 16 rows per CTA   (B, boxes of MAXT rows)
   const bf16* hidden;
   bf16* residual;
@@ -128,6 +136,7 @@ struct FusedParams {
   const bf16* norm_w;
   const bf16* gate_w;
   const float* gate_bias;
+  int w8;  // FP8 experts at one token, at most one routed unit per CTA: W8A8 (the note at kSharedUnit)
   const float* up_scale;    // [E, I] FP8 routed experts' row scales (else null)
   const float* down_scale;  // [E, H]
   int T, H, E, k, I, S;
@@ -205,6 +214,21 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Eight floats as E4M3 (round to nearest even, saturating), in order.
+__device__ __forceinline__ uint2 e4m3x8(const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h)
+    w[h] = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * h], v[2 * h + 1]), __NV_SATFINITE, __NV_E4M3);
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
 // Shared state of one CTA.
 struct Shared {
   uint64_t full[kStages], empty[kStages];
@@ -227,6 +251,8 @@ struct Shared {
   int U;                    // routed slots
   float rs[kDecodeMaxT];
   float red[4][kDecodeMaxT * 3];
+  float amax8[4];           // W8A8: per-warp maxima (token row, then relu^2 rows)
+  float x8s, u8s;           // W8A8: the E4M3 scales of the token row and of the relu^2 rows
   int seg_expert[kMaxSlots];            // expert of routed slot s
   float seg_w[kMaxSlots][kDecodeN];     // routing weight of token t in slot s (0 = not routed)
   int sel_idx[kDecodeMaxT * kTopKMax];
@@ -485,8 +511,9 @@ __device__ __forceinline__ void route_tokwarp(const FusedParams& p, Shared& sh, 
 }
 
 // One to four tokens (see RouteLoads); with one or two, from the loads
-// route_issue made.
-template <int MAXT>
+// route_issue made.  F8: the launch has FP8 routed experts (only then may
+// it write the E4M3 token row of W8A8).
+template <int MAXT, bool F8>
 __device__ void route_hold(const FusedParams& p, Shared& sh, int rt, RouteLoads<MAXT>& L,
                            bool f16tok) {
   const int H = p.H, T = p.T, E = p.E, G = gridDim.x;
@@ -560,6 +587,22 @@ __device__ void route_hold(const FusedParams& p, Shared& sh, int rt, RouteLoads<
       sh.red[warp][2 * MAXT + t] = v2;
     }
   }
+  // W8A8 (one token, FP8 units): the E4M3 copy of x * w needs the row's
+  // maximum |x * w| first
+  const bool want8 = F8 && f16tok && p.w8;
+  if constexpr (F8 && RouteLoads<MAXT>::kHold) if (want8) {
+    float xm = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxChunks; ++j) {
+      float f[8], g[8];
+      unpack8(L.x[j][0], f);
+      unpack8(L.w[j], g);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) xm = fmaxf(xm, fabsf(f[q] * g[q]));  // (zeros past H)
+    }
+    xm = warp_max(xm);
+    if (lane == 0) sh.amax8[warp] = xm;
+  }
   // the token rows: generic writes -> the TMA loads of this CTA's producer
   fence_proxy_async_global();
   named_barrier(kBarRoute, kRouteThreads);
@@ -567,6 +610,26 @@ __device__ void route_hold(const FusedParams& p, Shared& sh, int rt, RouteLoads<
   // weight stream may start.  Routing decides when the routed weights can
   // stream, so its loads go first.
   if (rt == 0) mbar_arrive(&sh.loads_out);
+  if constexpr (F8 && RouteLoads<MAXT>::kHold) if (want8) {
+    const float mx = fmaxf(fmaxf(sh.amax8[0], sh.amax8[1]), fmaxf(sh.amax8[2], sh.amax8[3]));
+    const float s8 = mx > 0.f ? mx / 448.f : 1.f;
+    const float inv = 1.f / s8;
+    if (rt == 0) sh.x8s = s8;
+    uint2* x8 = reinterpret_cast<uint2*>(p.ws.x8 + size_t(blockIdx.x) * kDecodeN * H);
+#pragma unroll
+    for (int j = 0; j < kMaxChunks; ++j) {
+      const int c = rt + j * kRouteThreads;
+      if (c < nv) {
+        float f[8], g[8];
+        unpack8(L.x[j][0], f);
+        unpack8(L.w[j], g);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] = f[q] * g[q] * inv;
+        x8[c] = e4m3x8(f);
+      }
+    }
+    fence_proxy_async_global();  // (the E4M3 row -> this CTA's TMA loads)
+  }
   if (rt < T) {
     float s = 0.f, a = 0.f, b = 0.f;
     for (int w = 0; w < 4; ++w) {
@@ -591,13 +654,13 @@ __device__ void route_hold(const FusedParams& p, Shared& sh, int rt, RouteLoads<
 // The routing pass of the routing warps (see RouteLoads).  f16tok: write the
 // token rows as f16 instead of BF16 (the up GEMM of FP8 units runs on f16
 // operands).
-template <int MAXT>
+template <int MAXT, bool F8>
 __device__ __forceinline__ void route_logits(const FusedParams& p, Shared& sh, int rt,
                                              RouteLoads<MAXT>& L, bool f16tok) {
   if constexpr (RouteLoads<MAXT>::kTokWarp)
     route_tokwarp<MAXT>(p, sh, rt, f16tok);
   else
-    route_hold<MAXT>(p, sh, rt, L, f16tok);
+    route_hold<MAXT, F8>(p, sh, rt, L, f16tok);
 }
 
 // The sigmoid top-k of token t by one warp, into sel_idx / sel_w.  The dry
@@ -995,7 +1058,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     if (F8) {
       for (int s = 0; s < kF8Slots; ++s) {
         mbar_init(&sh.f8full[s], 1);
-        mbar_init(&sh.f8empty[s], kRouteThreads / 32);  // freed by the four routing warps
+        // freed by the four dequantising warps, or under W8A8 by the MMA
+        mbar_init(&sh.f8empty[s], p.w8 ? 1 : kRouteThreads / 32);
       }
     }
     sh.abort = 0;
@@ -1009,6 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     tma_prefetch_desc(&p.tm_down);
     tma_prefetch_desc(&p.tm_sdown);
     tma_prefetch_desc(&p.tm_up64);
+    tma_prefetch_desc(&p.tm_x8);
     tma_prefetch_desc(&p.tm_sup64);
     tma_prefetch_desc(&p.tm_x);
   }
@@ -1123,9 +1188,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           tok8 = true;
         }
         uint8_t* sl = slots + fs * kF8SlotBytes;
-        mbar_arrive_expect_tx(&sh.f8full[fs], uint32_t(kF8ABytes + (up ? kKB * MAXT * 128 : 0)));
+        // (the up's token rows: two f16 boxes for the dequantising path, one
+        // E4M3 box of the same 128 elements under W8A8)
+        mbar_arrive_expect_tx(&sh.f8full[fs],
+                              uint32_t(kF8ABytes + (up ? (p.w8 ? 1 : kKB) * MAXT * 128 : 0)));
         tma_load_2d_hint(sl, map, &sh.f8full[fs], ax, ay, stream_policy);
-        if (up)
+        if (up && p.w8)
+          tma_load_2d(sl + kF8ABytes, &p.tm_x8, &sh.f8full[fs], bx, xrow);
+        else if (up)
           for (int i = 0; i < kKB; ++i)
             tma_load_2d(sl + kF8ABytes + i * kBBytes, &p.tm_x, &sh.f8full[fs], bx + i * 64, xrow);
         ++issued8;
@@ -1236,6 +1306,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     if (lane == 0) {
       const uint32_t idesc = make_idesc(kBM, kDecodeN, 1, 1);    // BF16 x BF16 -> F32
       const uint32_t idesc_h = make_idesc(kBM, kDecodeN, 0, 0);  // F16 x F16 -> F32 (FP8 units' up)
+      const uint32_t idesc_8 = make_idesc(kBM, kDecodeN, 0, 0);  // E4M3 x E4M3 -> F32 (W8A8)
+      const bool w8 = conv && p.w8;  // (W8A8: the MMA reads the FP8 slots themselves)
+      const uint8_t* slots = tiles + kStagesF8 * kStageBytes;
+      int fs = 0;
+      uint32_t fph = 0;
+      // the next FP8 slot, once its boxes have landed; false on timeout
+      auto slot_wait = [&]() -> bool {
+        if (!mbar_wait(&sh.f8full[fs], fph, abort)) {
+          record_timeout(p.status, abort);
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      auto slot_release = [&]() {
+        umma_commit(&sh.f8empty[fs]);
+        if (++fs == kF8Slots) {
+          fs = 0;
+          fph ^= 1u;
+        }
+      };
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -1268,6 +1359,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           }
           tc_fence_after();
           const uint32_t d = tmem_base + uint32_t(b * kDecodeN);
+          if (w8) {  // one slot per two k-blocks: 128 E4M3 weights x 128 E4M3 token bytes
+            for (int kb = 0; ok && kb < kbH; kb += kKB) {
+              if (!slot_wait()) {
+                ok = false;
+                break;
+              }
+              const uint8_t* sl = slots + fs * kF8SlotBytes;
+              const uint64_t ad = smem_desc_sw128(sl);
+              const uint64_t bd = smem_desc_sw128(sl + kF8ABytes);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t koff = uint64_t((kk * 32) >> 4);
+                umma_f8(d, ad + koff, bd + koff, idesc_8, (kb != 0 || kk != 0) ? 1u : 0u);
+              }
+              slot_release();
+            }
+            if (ok) umma_commit(&sh.tfull[b]);
+            continue;
+          }
           for (int kb = 0; kb < kbH; kb += kKB) {
             if (!mbar_wait(&sh.full[stage], phase, abort)) {
               record_timeout(p.status, abort);
@@ -1304,6 +1414,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           }
           tc_fence_after();
           const uint8_t* ub = ubufs + b * kUBytes;
+          if (w8) {  // the unit's 128 K columns of each 128-row block of H in one slot
+            for (int r = 0; ok && r < nH; ++r) {
+              const uint32_t d = tmem_base + uint32_t((2 + r) * kDecodeN);
+              if (!slot_wait()) {
+                ok = false;
+                break;
+              }
+              const uint64_t ad = smem_desc_sw128(slots + fs * kF8SlotBytes);
+              const uint64_t bd = smem_desc_sw128(ub);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t koff = uint64_t((kk * 32) >> 4);
+                umma_f8(d, ad + koff, bd + koff, idesc_8, (n != 0 || kk != 0) ? 1u : 0u);
+              }
+              slot_release();
+            }
+            if (ok) umma_commit(&sh.ufree[b]);
+            continue;
+          }
           const int nkk = down_kk(f);
           for (int r = 0; ok && r < nH; ++r) {
             const uint32_t d = tmem_base + uint32_t((2 + r) * kDecodeN);
@@ -1358,6 +1487,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     // the tokens this CTA's units reach: its partial output is exactly zero
     // in every other column (their relu^2 rows are zero), which it need not add
     uint32_t tmask = 0;
+    const bool w8 = conv && p.w8;
+    int e8 = 0;  // (W8A8: the expert of the CTA's one unit)
     for (int n = 0; ok; ++n) {
       if (n >= m) {
         if (routed) break;
@@ -1376,6 +1507,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       const UnitInfo f = unit_info(p, sh, un, n);
       const int b = n & 1;
       const uint32_t par = (n >> 1) & 1;
+      e8 = f.expert;
 #pragma unroll
       for (int c = 0; c < MAXT; ++c)
         if (c < p.T && (f.shared || sh.seg_w[f.slot][c] != 0.f)) tmask |= 1u << c;
@@ -1402,11 +1534,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       // relu^2 times the routing weight (1 for the shared expert); rows past
       // the matrix (an expert's last tile) and tokens past T are zero
       float v[kDecodeN];
+      const float s8 = w8 ? sh.x8s : 1.f;  // (W8A8: the token row's E4M3 scale)
 #pragma unroll
       for (int c = 0; c < kDecodeN; ++c) {
         const float w = f.shared ? (c < p.T ? 1.f : 0.f) : sh.seg_w[f.slot][c];
-        const float a = __uint_as_float(r[c]) * rsc[c] * srow;
+        const float a = __uint_as_float(r[c]) * rsc[c] * srow * s8;
         v[c] = valid && w != 0.f ? (a > 0.f ? a * a : 0.f) * w : 0.f;
+      }
+      // W8A8 (one token): the relu^2 rows as E4M3 with one scale, max |v| / 448
+      float inv8 = 1.f;
+      if (w8) {
+        const float um = warp_max(fabsf(v[0]));
+        if (lane == 0) sh.amax8[warp & 3] = um;
+        named_barrier(kBarEpi, kEpiThreads);
+        const float mx = fmaxf(fmaxf(sh.amax8[0], sh.amax8[1]), fmaxf(sh.amax8[2], sh.amax8[3]));
+        const float su = mx > 0.f ? mx / 448.f : 1.f;
+        inv8 = 1.f / su;
+        if (tid == 0) sh.u8s = su;
       }
       // buffer b is free once unit n - 2's down MMAs have completed
       if (n >= 2) {
@@ -1418,7 +1562,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
           break;
         }
       }
-      store_u_row(ubufs + b * kUBytes, rloc, v);
+      if (w8) {
+        // K-major E4M3 token rows of 128 bytes (128-byte swizzle: 16-byte chunk
+        // j of row c at j ^ (c % 8)); row 0 is the token, the others zero
+        uint8_t* ub = ubufs + b * kUBytes;
+        const __nv_fp8x2_storage_t q2 = __nv_cvt_float2_to_fp8x2(
+            make_float2(v[0] * inv8, 0.f), __NV_SATFINITE, __NV_E4M3);
+#pragma unroll
+        for (int c = 0; c < kDecodeN; ++c)
+          ub[c * 128 + ((((rloc >> 4) ^ (c & 7)) << 4) | (rloc & 15))] =
+              c == 0 ? uint8_t(q2 & 0xffu) : uint8_t(0);
+      } else {
+        store_u_row(ubufs + b * kUBytes, rloc, v);
+      }
       fence_proxy_async_shared();  // generic writes -> tensor core reads
       named_barrier(kBarEpi, kEpiThreads);
       if (tid == 0) mbar_arrive(&sh.ufull[b]);
@@ -1461,10 +1617,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
 #pragma unroll
             for (int c = 0; c < MAXT; ++c) {
               if (!((tmask >> c) & 1u)) continue;
+              // (W8A8: the down weight row's scale and the relu^2 rows' scale)
+              const float sc8 =
+                  w8 ? p.down_scale[size_t(e8) * p.H + row] * sh.u8s : 1.f;
               if constexpr (kStagePartial)
-                stagef[c * p.H + row] = __uint_as_float(r[g][c]);
+                stagef[c * p.H + row] = __uint_as_float(r[g][c]) * sc8;
               else
-                add_partial(p.ws, size_t(c) * p.H + row, __uint_as_float(r[g][c]));
+                add_partial(p.ws, size_t(c) * p.H + row, __uint_as_float(r[g][c]) * sc8);
             }
           }
         }
@@ -1482,10 +1641,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   } else {
     // ------------------------------------------------------------- routing
     const int rt = threadIdx.x - 192;
-    route_logits<MAXT>(p, sh, rt, rl, conv);
+    route_logits<MAXT, F8>(p, sh, rt, rl, conv);
     const bool routed_ok = route_select(p, sh, rt, abort, kBarRoute, false);
     if (rt == 0) mbar_arrive(&sh.routed);  // (also on failure: the waiters then see abort)
-    if (conv && routed_ok && !*abort) {
+    if (conv && !p.w8 && routed_ok && !*abort) {
       Units ur = un;
       ur.N = un.nS + sh.U * un.nI;
       dequant_stages(p, sh, ur, tiles, rt, abort);
@@ -1600,6 +1759,7 @@ cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   p.tm_down = *a.tm_down;
   p.tm_sdown = *a.tm_sdown;
   p.tm_up64 = *a.tm_up64;
+  p.tm_x8 = *a.tm_x8;
   p.tm_sup64 = *a.tm_sup64;
   const int bucket = a.T <= 1 ? 0 : a.T <= 2 ? 1 : a.T <= 4 ? 2 : 3;
   p.tm_x = *a.tm_x[bucket];
@@ -1621,6 +1781,13 @@ cudaError_t launch_fused_decode(const FusedDecodeArgs& a, cudaStream_t stream) {
   p.rsf = c.routed_scaling_factor;
   p.ws = *a.ws;
   p.status = a.status;
+  // W8A8 (the note at kSharedUnit): one token chooses top_k distinct
+  // experts; their routed units must fit on the CTAs beside the shared ones
+  {
+    const int nS = (c.shared_inter + kSharedUnit - 1) / kSharedUnit;
+    const int nI = (c.moe_inter + kBM - 1) / kBM;
+    p.w8 = f8 && a.T == 1 && c.top_k * nI <= a.grid - nS ? 1 : 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.grid);
   cfg.blockDim = dim3(kThreads);

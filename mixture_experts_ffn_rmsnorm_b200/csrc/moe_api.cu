@@ -156,6 +156,7 @@ struct moe_handle {
   int up_bn, down_bn;
   CUtensorMap tm_fc2_a, tm_fc2_b;
   CUtensorMap tm_dec_x[4];  // decode token rows, one 16-row block per CTA; boxes of 1, 2, 4, 8 rows
+  CUtensorMap tm_dec_x8;    // the E4M3 token rows of the one-token FP8 launch, one-row boxes
 };
 
 namespace {
@@ -332,10 +333,12 @@ bool build_maps(moe_handle* h) {
   ok &= make_map(&h->tm_sup_w, h->w.shared_up_w, sf8, H, S, H * sb, h->up_bn);
   ok &= make_map(&h->tm_down_w, h->w.down_w, f8, I, E * D, I * eb, h->down_bn);
   ok &= make_map(&h->tm_sdown_w, h->w.shared_down_w, sf8, S, H, S * sb, h->down_bn);
-  if (moe::fused_decode_supported(c, h->num_sms))
+  if (moe::fused_decode_supported(c, h->num_sms)) {
     for (int b = 0; b < 4; ++b)
       ok &= make_map(&h->tm_dec_x[b], h->dec.x16, false, H, uint64_t(h->num_sms) * moe::kDecodeN,
                      H * 2, 1u << b);
+    ok &= make_map(&h->tm_dec_x8, h->dec.x8, true, H, uint64_t(h->num_sms) * moe::kDecodeN, H, 1);
+  }
   return ok;
 }
 
@@ -585,6 +588,7 @@ moe_status enqueue_decode(moe_handle* h, bf16* hidden, bf16* residual, int T, cu
   a.tm_up64 = &h->tm_up_b64;  // the same up weights, 64-row boxes
   a.tm_sup64 = &h->tm_sup_b64;
   for (int b = 0; b < 4; ++b) a.tm_x[b] = &h->tm_dec_x[b];
+  a.tm_x8 = &h->tm_dec_x8;
   a.hidden = hidden;
   a.residual = residual;
   a.out = out;
