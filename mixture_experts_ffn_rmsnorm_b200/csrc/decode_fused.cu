@@ -37,6 +37,8 @@
 //              operand); CTA 0 writes the residual.  Once every CTA's logits
 //              are in, each CTA runs the same sigmoid top-k and builds the
 //              same table of routed slots (distinct experts, first-use order).
+//              With FP8 routed units they then dequantise the weight boxes
+//              (or, W8A8 at one token, write an E4M3 copy of the token row).
 //   all        the final reduction.
 //
 // Every wait is bounded (about one second): a timeout sets a status bit, the
@@ -232,7 +234,7 @@ __device__ __forceinline__ uint2 e4m3x8(const float (&v)[8]) {
 // Shared state of one CTA.
 struct Shared {
   uint64_t full[kStages], empty[kStages];
-  uint64_t f8full[kF8Slots], f8empty[kF8Slots];  // FP8 staging slots: TMA -> dequantisation
+  uint64_t f8full[kF8Slots], f8empty[kF8Slots];  // FP8 staging slots: TMA -> dequantisation (or MMA, W8A8)
   uint64_t tfull[2], tempty[2];   // up accumulators: MMA -> epilogue -> MMA
   uint64_t ufull[2], ufree[2];    // relu^2 row buffers: epilogue -> MMA -> epilogue
   uint64_t down_done;             // every down MMA of the CTA has completed
@@ -1029,7 +1031,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   un.nI = (p.I + kBM - 1) / kBM;
   un.N = un.nS;  // the routed units are added once the routing is known
   un.f8 = F8;
-  // this CTA's units are FP8 (dequantised by the routing warps), and the
+  // this CTA's units are FP8 (dequantised by the routing warps, or read by the MMA under W8A8), and the
   // BF16 stages it has
   const bool conv = F8 && cta >= un.nS;
   const int nst = conv ? kStagesF8 : kStages;

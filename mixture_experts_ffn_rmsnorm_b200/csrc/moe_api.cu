@@ -562,10 +562,11 @@ moe_status enqueue_prefill(moe_handle* h, bf16* hidden, bf16* residual, int T, c
 // Decode path (T <= 8): one cooperative launch (decode_fused.cu) with the
 // weights as the 128-row operand and the tokens as N = 16.
 // Whether MOE_PATH_AUTO takes the decode launch.  With FP8 routed experts
-// only one token does: the launch then dequantises the weights in shared
-// memory, which pays while every routed unit has a CTA to itself (one
-// token) and not beyond (measured on B200 with the skewed FP8 workload's
-// layer: 75 against 98 us at T = 1, 118 against 104 us at T = 2).
+// only one token does: there every routed unit has a CTA to itself, and the
+// launch runs W8A8 on the E4M3 weights (47 us on B200 for the skewed FP8
+// workload's layer, against 98 us on the prefill path).  From two tokens
+// on it dequantises the weights in shared memory, which no longer pays
+// (118 against 104 us at T = 2).
 bool decode_preferred(const moe_handle* h, int T) {
   return T <= MOE_DECODE_MAX_TOKENS && moe::fused_decode_supported(h->cfg, h->num_sms) &&
          (h->cfg.expert_wdtype == MOE_WEIGHTS_BF16 || T == 1);
